@@ -1,0 +1,54 @@
+"""The oracle pins must catch plausible mistakes.
+
+Each case copies oracle/veda_oracle.c, plants one mistake (a dropped term, a
+wrong index, a reversed comparison, ...), compiles the copy on the CPU and runs
+the pin suite against it: the suite has to fail.  The committed oracle is
+never modified.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "veda_oracle.c")
+
+MUTANTS = {
+    "pool_divides_by_T": ("o[e] = o[e] / (double)c;", "o[e] = o[e] / (double)T;"),
+    "pool_tile_end_off_by_one": ("int64_t t1 = min64(N, t0 + T);", "int64_t t1 = min64(N, t0 + T - 1);"),
+    "project_transposed_weight": ("(h * d + e) * r + c)", "(h * r + c) * d + e)"),
+    "project_ignores_head": ("(h * d + e) * r + c)", "(e) * r + c)"),
+    "score_uses_query_twice": ("acc += q[c] * k[c];", "acc += q[c] * q[c];"),
+    "select_keeps_lowest_scores": ("if (a->s > b->s) return -1;\n    if (a->s < b->s) return 1;",
+                                   "if (a->s < b->s) return -1;\n    if (a->s > b->s) return 1;"),
+    "select_ties_to_highest_index": ("return (a->j > b->j) - (a->j < b->j);",
+                                     "return (a->j < b->j) - (a->j > b->j);"),
+    "select_output_not_ascending": ("qsort(dst, (size_t)k, sizeof(int32_t), int32_ascending);", ""),
+    "attend_drops_dense_keys": ("for (int64_t t = 0; t < p->dense.n; ++t) {",
+                                "for (int64_t t = 0; t < 0; ++t) {"),
+    "attend_reference_uses_video_index": ("int64_t j = idx_r[rid * k_r + m];",
+                                          "int64_t j = idx_v[rid * k_v + m];"),
+    "attend_forgets_scale": ("logit[a] = p->scale * dot;", "logit[a] = dot;"),
+    "attend_logits_against_values": ("dot += qrow[e] * elem(s->k, p->dtype, base + e);",
+                                     "dot += qrow[e] * elem(s->v, p->dtype, base + e);"),
+    "attend_no_max_subtraction": ("const double w = exp(logit[a] - mx);", "const double w = exp(logit[a]);"),
+    "attend_unnormalised": ("for (int64_t e = 0; e < d; ++e) o[e] = o[e] / z;", ""),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    mutant = tmp_path / "mutant.c"
+    mutant.write_text(src.replace(old, new))
+    so = tmp_path / "libmutant.so"
+    subprocess.run(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-ffp-contract=off",
+                    "-o", str(so), str(mutant), "-lm"], check=True)
+    env = dict(os.environ, VEDA_ORACLE_LIB=str(so), OMP_NUM_THREADS="2")
+    res = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                          os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                         cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert res.returncode != 0, f"pins did not catch mutant {name}:\n{res.stdout[-2000:]}"
