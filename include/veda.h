@@ -1,0 +1,181 @@
+/*
+ * veda.h -- C ABI of libveda: Veda-style learned block-sparse attention for
+ * video diffusion transformers on NVIDIA B200 (sm_100a).
+ *
+ * What the library computes (the pages state it in prose only):
+ *   1. Tile pooling + selector projection.  A lightweight predictor scores
+ *      blocks of the attention map; its trainable parts are a query and a key
+ *      projection per layer, applied to tile-pooled Q and K (tao.media,
+ *      "Affine launches MiniMax-H3 video studio and SN120 sparse attention
+ *      competition", sections "Training the Selector, Not the Generator" and
+ *      "How the SN120 Competition Works").  Pooling = the mean over the
+ *      tokens that exist in a tile (a short last tile is averaged over its
+ *      own tokens); projection = pooled row vector times W[h] ([d, r]).
+ *   2. Tile scoring: s[i][j] = qhat_i . khat_j (raw dot product).
+ *   3. Fixed-budget selection: per (batch, head, query tile) keep the
+ *      `budget` key tiles of highest score, ties to the lowest tile index,
+ *      emitted in ascending order (budgets: same article, section "How the
+ *      SN120 Competition Works"; 32 reference + 32 video tiles chosen
+ *      independently: veyrul.com, "Veda R2VA for MiniMax-H3", second
+ *      paragraph).
+ *   4. Block-sparse attention: each video query attends to every token of
+ *      its query tile's kept video tiles, kept reference tiles, and every
+ *      dense (text / VLM / audio) token, with one softmax over that set
+ *      (same veyrul.com paragraph: text, VLM and audio attention stay dense).
+ *      Tokens past the end of a segment are not keys.
+ *
+ * Conventions (all entry points):
+ *   - Every pointer argument except `ws` sizes is a DEVICE pointer owned by
+ *     the caller; the library allocates no device memory and keeps no mutable
+ *     global state, so concurrent calls on different workspaces are safe.
+ *   - All work is enqueued on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream); calls return after enqueueing, without synchronising.
+ *   - Argument errors are detected on the host before anything is launched
+ *     and returned synchronously.  Errors found on the device (an index out
+ *     of range, a bounded wait that ran out) are recorded in a sticky status
+ *     word inside the workspace and returned by veda_check_status().
+ *   - Layouts: activations are [B, n_tokens, H, d] with d contiguous and the
+ *     other three strides given in ELEMENTS; every base pointer must be
+ *     16-byte aligned and every stride * element size a multiple of 16 bytes.
+ *     Selector weights are contiguous [H, d, r] in the problem's dtype.
+ *     Kept-tile indices are contiguous int32 [B, H, n_q_tiles, budget].
+ *     The attention output is contiguous [B, n_video_tokens, H, d] in the
+ *     problem's dtype; the optional log-sum-exp is contiguous fp32
+ *     [B, H, n_video_tokens] (natural log, of the scaled logits).
+ */
+#ifndef VEDA_H
+#define VEDA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define VEDA_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define VEDA_API __attribute__((visibility("default")))
+#else
+#define VEDA_API
+#endif
+
+typedef struct CUstream_st* veda_stream_t; /* == cudaStream_t */
+
+typedef enum {
+    VEDA_OK = 0,
+    VEDA_ERR_INVALID_ARG = -1,  /* bad pointer, size, stride, alignment or budget      */
+    VEDA_ERR_UNSUPPORTED = -2,  /* valid but not implemented (d, tile, r, dtype, size) */
+    VEDA_ERR_WORKSPACE = -3,    /* workspace NULL, misaligned or too small             */
+    VEDA_ERR_CUDA = -4,         /* a CUDA launch or driver call failed                 */
+    VEDA_ERR_TIMEOUT = -5,      /* device: a bounded wait ran out (kernel returned)    */
+    VEDA_ERR_BAD_INDEX = -6     /* device: a kept-tile index was outside its segment   */
+} veda_status;
+
+typedef enum { VEDA_F32 = 0, VEDA_BF16 = 1 } veda_dtype;
+
+/* Problem flags. */
+#define VEDA_FLAG_SIMT_ATTENTION 1u /* run attention on the fp32 SIMT kernel even
+                                       where the tensor-core kernel applies (bf16,
+                                       d = 128, tile = 128): a cross-check path  */
+
+/* One key/value segment, [B, n_tokens, H, d] (d contiguous). */
+typedef struct {
+    const void* k;
+    const void* v;
+    int64_t n_tokens;   /* 0: segment absent (ref / dense only) */
+    int64_t stride_b;   /* element strides of k and v (shared) */
+    int64_t stride_tok;
+    int64_t stride_h;
+    int32_t budget;     /* sparse segments: kept tiles per (query tile, head),
+                           1 <= budget <= ceil(n_tokens / tile).
+                           dense segment: must be 0. */
+    int32_t reserved;
+} veda_segment;
+
+/* One attention layer call.  Queries are the video tokens (q has
+ * video.n_tokens tokens); query tile i covers the same tokens as video key
+ * tile i. */
+typedef struct {
+    int32_t B, H;
+    int32_t d;          /* head dim: 64 or 128 */
+    int32_t tile;       /* tokens per tile (query and key): 64 or 128 */
+    int32_t r;          /* selector width: 1..128, multiple of 4 */
+    veda_dtype dtype;   /* of q, k, v, weights and output */
+    float softmax_scale;/* 0: 1/sqrt(d) */
+    uint32_t flags;     /* VEDA_FLAG_* */
+    const void* q;
+    int64_t q_stride_b, q_stride_tok, q_stride_h;
+    veda_segment video; /* sparse, required */
+    veda_segment ref;   /* sparse visual-reference segment, optional */
+    veda_segment dense; /* always-attended text / VLM / audio keys, optional */
+} veda_problem;
+
+/* Bytes of device workspace the calls below need for this problem (pooled
+ * projections, tile scores and the status word).  The workspace must be
+ * 256-byte aligned and prepared once with veda_workspace_init(). */
+VEDA_API veda_status veda_workspace_size(const veda_problem* p, size_t* bytes);
+
+/* Zero the workspace's status word (enqueued on `stream`).  Call once after
+ * allocating a workspace; veda_check_status() re-arms it after each read. */
+VEDA_API veda_status veda_workspace_init(void* ws, size_t ws_bytes, veda_stream_t stream);
+
+/* Steps 1-3: pool + project Q and K, score every key tile, keep the top
+ * `budget` per (b, h, query tile) for the video segment and, when present,
+ * independently for the reference segment.
+ *   w_q, w_k   [H, d, r] device, problem dtype
+ *   idx_video  [B, H, n_q_tiles, video.budget] int32 out (ascending rows)
+ *   idx_ref    [B, H, n_q_tiles, ref.budget]   int32 out; NULL iff no reference */
+VEDA_API veda_status veda_select_tiles(const veda_problem* p, const void* w_q, const void* w_k,
+                              int32_t* idx_video, int32_t* idx_ref,
+                              void* ws, size_t ws_bytes, veda_stream_t stream);
+
+/* Step 4: attention over the caller's kept tiles plus every dense token.
+ *   idx_video / idx_ref: as produced by veda_select_tiles (any order is
+ *   accepted; an index outside its segment is skipped and flagged as
+ *   VEDA_ERR_BAD_INDEX in the status word).
+ *   out [B, video.n_tokens, H, d] problem dtype; lse [B, H, video.n_tokens]
+ *   fp32 or NULL. */
+VEDA_API veda_status veda_block_sparse_attn(const veda_problem* p, const int32_t* idx_video,
+                                   const int32_t* idx_ref, void* out, float* lse,
+                                   void* ws, size_t ws_bytes, veda_stream_t stream);
+
+/* Steps 1-4 in one call (selection, then attention on the selected tiles),
+ * stream-ordered, no host synchronisation.  idx_video / idx_ref receive the
+ * kept tiles as in veda_select_tiles. */
+VEDA_API veda_status veda_attn(const veda_problem* p, const void* w_q, const void* w_k,
+                      int32_t* idx_video, int32_t* idx_ref, void* out, float* lse,
+                      void* ws, size_t ws_bytes, veda_stream_t stream);
+
+/* The three stages of veda_select_tiles, exposed for timing and testing.
+ * They communicate through the workspace; call them in this order. */
+/* Step 1 for Q, video K and (if present) reference K. */
+VEDA_API veda_status veda_pool_project(const veda_problem* p, const void* w_q, const void* w_k,
+                              void* ws, size_t ws_bytes, veda_stream_t stream);
+/* Step 2: fp32 tile scores of every sparse segment into the workspace. */
+VEDA_API veda_status veda_score_tiles(const veda_problem* p, void* ws, size_t ws_bytes,
+                             veda_stream_t stream);
+/* Step 3: top-k of the workspace scores into idx_video / idx_ref. */
+VEDA_API veda_status veda_topk_tiles(const veda_problem* p, int32_t* idx_video, int32_t* idx_ref,
+                            void* ws, size_t ws_bytes, veda_stream_t stream);
+
+/* Read-only views of the workspace (device pointers), for tests:
+ *   which = 0: qhat [B,H,n_q_tiles,r] fp32     1: khat video [B,H,n_q_tiles,r]
+ *           2: khat ref [B,H,n_ref_tiles,r]    3: scores video [B,H,n_q_tiles,ld]
+ *           4: scores ref [B,H,n_q_tiles,ld]
+ * *ld receives the row stride (elements) of the score matrices (>= n tiles). */
+VEDA_API veda_status veda_workspace_view(const veda_problem* p, void* ws, size_t ws_bytes, int which,
+                                const void** ptr, int64_t* ld);
+
+/* Synchronise `stream`, return the sticky device status recorded in `ws`
+ * since the last check (VEDA_OK if none), and reset it. */
+VEDA_API veda_status veda_check_status(void* ws, veda_stream_t stream);
+
+/* Static, human-readable name of a status code. */
+VEDA_API const char* veda_status_string(veda_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* VEDA_H */

@@ -1,0 +1,234 @@
+"""ctypes binding of libveda (include/veda.h): argument marshalling only.
+
+Every step of the computation runs in the CUDA library; this module only
+fills the C structs from torch tensors (device pointers, element strides) and
+passes the current CUDA stream.  There is no fallback: if libveda.so is
+missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libveda.so")
+
+VEDA_OK = 0
+VEDA_ERR_INVALID_ARG = -1
+VEDA_ERR_UNSUPPORTED = -2
+VEDA_ERR_WORKSPACE = -3
+VEDA_ERR_CUDA = -4
+VEDA_ERR_TIMEOUT = -5
+VEDA_ERR_BAD_INDEX = -6
+VEDA_F32, VEDA_BF16 = 0, 1
+VEDA_FLAG_SIMT_ATTENTION = 1
+
+EXPORTS = ("veda_workspace_size", "veda_workspace_init", "veda_select_tiles", "veda_block_sparse_attn",
+           "veda_attn", "veda_pool_project", "veda_score_tiles", "veda_topk_tiles", "veda_workspace_view",
+           "veda_check_status", "veda_status_string")
+
+
+class VedaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+        self.status = status
+
+
+class veda_segment(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("n_tokens", ctypes.c_int64),
+                ("stride_b", ctypes.c_int64), ("stride_tok", ctypes.c_int64), ("stride_h", ctypes.c_int64),
+                ("budget", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+class veda_problem(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("d", ctypes.c_int32), ("tile", ctypes.c_int32),
+                ("r", ctypes.c_int32), ("dtype", ctypes.c_int32), ("softmax_scale", ctypes.c_float),
+                ("flags", ctypes.c_uint32), ("q", ctypes.c_void_p), ("q_stride_b", ctypes.c_int64),
+                ("q_stride_tok", ctypes.c_int64), ("q_stride_h", ctypes.c_int64),
+                ("video", veda_segment), ("ref", veda_segment), ("dense", veda_segment)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libveda.so; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m learned_block_sparse_pool_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P = ctypes.POINTER(veda_problem)
+        vp, sz, i32p = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p
+        L.veda_workspace_size.argtypes = [P, ctypes.POINTER(ctypes.c_size_t)]
+        L.veda_workspace_init.argtypes = [vp, sz, vp]
+        L.veda_select_tiles.argtypes = [P, vp, vp, i32p, i32p, vp, sz, vp]
+        L.veda_block_sparse_attn.argtypes = [P, i32p, i32p, vp, vp, vp, sz, vp]
+        L.veda_attn.argtypes = [P, vp, vp, i32p, i32p, vp, vp, vp, sz, vp]
+        L.veda_pool_project.argtypes = [P, vp, vp, vp, sz, vp]
+        L.veda_score_tiles.argtypes = [P, vp, sz, vp]
+        L.veda_topk_tiles.argtypes = [P, i32p, i32p, vp, sz, vp]
+        L.veda_workspace_view.argtypes = [P, vp, sz, ctypes.c_int, ctypes.POINTER(ctypes.c_void_p),
+                                          ctypes.POINTER(ctypes.c_int64)]
+        L.veda_check_status.argtypes = [vp, vp]
+        L.veda_status_string.argtypes = [ctypes.c_int]
+        L.veda_status_string.restype = ctypes.c_char_p
+        for name in EXPORTS:
+            if name != "veda_status_string":
+                getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def status_string(s: int) -> str:
+    return lib().veda_status_string(int(s)).decode()
+
+
+def _check(st: int, where: str) -> None:
+    if st != VEDA_OK:
+        raise VedaError(st, where)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return VEDA_BF16
+    if t.dtype == torch.float32:
+        return VEDA_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+class Problem:
+    """A veda_problem plus references to the tensors it points at."""
+
+    def __init__(self, q, k, v, *, tile: int, r: int, budget: int, k_ref=None, v_ref=None,
+                 budget_ref: int = 0, k_dense=None, v_dense=None, scale: float = 0.0, flags: int = 0):
+        B, N, H, d = q.shape
+        self.tensors = [q, k, v, k_ref, v_ref, k_dense, v_dense]
+        c = veda_problem()
+        c.B, c.H, c.d, c.tile, c.r = B, H, d, tile, r
+        c.dtype = _dtype_code(q)
+        c.softmax_scale = float(scale)
+        c.flags = int(flags)
+        c.q = q.data_ptr()
+        c.q_stride_b, c.q_stride_tok, c.q_stride_h = q.stride(0), q.stride(1), q.stride(2)
+        self._seg(c.video, k, v, budget)
+        self._seg(c.ref, k_ref, v_ref, budget_ref)
+        self._seg(c.dense, k_dense, v_dense, 0)
+        self.c = c
+        self.B, self.H, self.d, self.tile, self.N = B, H, d, tile, N
+        self.n_q_tiles = -(-N // tile)
+        self.n_ref_tiles = 0 if k_ref is None else -(-k_ref.shape[1] // tile)
+        self.budget, self.budget_ref = budget, budget_ref
+        self.dtype = q.dtype
+        self.device = q.device
+
+    @staticmethod
+    def _seg(seg, k, v, budget):
+        if k is None:
+            seg.k = seg.v = None
+            seg.n_tokens = seg.stride_b = seg.stride_tok = seg.stride_h = 0
+            seg.budget = int(budget)
+            return
+        if k.stride() != v.stride() or k.shape != v.shape:
+            raise ValueError("k and v of a segment must share shape and strides")
+        seg.k, seg.v = k.data_ptr(), v.data_ptr()
+        seg.n_tokens = k.shape[1]
+        seg.stride_b, seg.stride_tok, seg.stride_h = k.stride(0), k.stride(1), k.stride(2)
+        seg.budget = int(budget)
+
+    @property
+    def has_ref(self) -> bool:
+        return self.c.ref.n_tokens > 0
+
+    def ref(self):
+        return ctypes.byref(self.c)
+
+
+def workspace_size(p: Problem) -> int:
+    n = ctypes.c_size_t()
+    _check(lib().veda_workspace_size(p.ref(), ctypes.byref(n)), "veda_workspace_size")
+    return n.value
+
+
+def workspace(p: Problem, stream=None) -> torch.Tensor:
+    """Allocate (with torch) and initialise a workspace for `p`."""
+    n = workspace_size(p)
+    ws = torch.empty(n, dtype=torch.uint8, device=p.device)
+    if ws.data_ptr() % 256:
+        raise RuntimeError("workspace allocation not 256-byte aligned")
+    _check(lib().veda_workspace_init(ws.data_ptr(), n, _stream(stream)), "veda_workspace_init")
+    return ws
+
+
+def alloc_indices(p: Problem) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    iv = torch.empty((p.B, p.H, p.n_q_tiles, p.budget), dtype=torch.int32, device=p.device)
+    ir = (torch.empty((p.B, p.H, p.n_q_tiles, p.budget_ref), dtype=torch.int32, device=p.device)
+          if p.has_ref else None)
+    return iv, ir
+
+
+def alloc_output(p: Problem, with_lse: bool = False):
+    out = torch.empty((p.B, p.N, p.H, p.d), dtype=p.dtype, device=p.device)
+    lse = torch.empty((p.B, p.H, p.N), dtype=torch.float32, device=p.device) if with_lse else None
+    return out, lse
+
+
+def select_tiles(p: Problem, w_q, w_k, idx_v, idx_r, ws, stream=None) -> None:
+    _check(lib().veda_select_tiles(p.ref(), w_q.data_ptr(), w_k.data_ptr(), _ptr(idx_v), _ptr(idx_r),
+                                   ws.data_ptr(), ws.numel(), _stream(stream)), "veda_select_tiles")
+
+
+def block_sparse_attn(p: Problem, idx_v, idx_r, out, lse, ws, stream=None) -> None:
+    _check(lib().veda_block_sparse_attn(p.ref(), _ptr(idx_v), _ptr(idx_r), out.data_ptr(), _ptr(lse),
+                                        ws.data_ptr(), ws.numel(), _stream(stream)), "veda_block_sparse_attn")
+
+
+def attn(p: Problem, w_q, w_k, idx_v, idx_r, out, lse, ws, stream=None) -> None:
+    _check(lib().veda_attn(p.ref(), w_q.data_ptr(), w_k.data_ptr(), _ptr(idx_v), _ptr(idx_r), out.data_ptr(),
+                           _ptr(lse), ws.data_ptr(), ws.numel(), _stream(stream)), "veda_attn")
+
+
+def pool_project(p: Problem, w_q, w_k, ws, stream=None) -> None:
+    _check(lib().veda_pool_project(p.ref(), w_q.data_ptr(), w_k.data_ptr(), ws.data_ptr(), ws.numel(),
+                                   _stream(stream)), "veda_pool_project")
+
+
+def score_tiles(p: Problem, ws, stream=None) -> None:
+    _check(lib().veda_score_tiles(p.ref(), ws.data_ptr(), ws.numel(), _stream(stream)), "veda_score_tiles")
+
+
+def topk_tiles(p: Problem, idx_v, idx_r, ws, stream=None) -> None:
+    _check(lib().veda_topk_tiles(p.ref(), _ptr(idx_v), _ptr(idx_r), ws.data_ptr(), ws.numel(),
+                                 _stream(stream)), "veda_topk_tiles")
+
+
+def workspace_view(p: Problem, ws, which: int) -> torch.Tensor:
+    """Copy-free view of a workspace region as a torch tensor (device)."""
+    ptr = ctypes.c_void_p()
+    ld = ctypes.c_int64()
+    _check(lib().veda_workspace_view(p.ref(), ws.data_ptr(), ws.numel(), which, ctypes.byref(ptr),
+                                     ctypes.byref(ld)), "veda_workspace_view")
+    n_rows_tiles = p.n_ref_tiles if which == 2 else p.n_q_tiles
+    shape = (p.B, p.H, n_rows_tiles, ld.value)
+    off = ptr.value - ws.data_ptr()
+    nbytes = 4 * p.B * p.H * n_rows_tiles * ld.value
+    return ws[off:off + nbytes].view(torch.float32).view(shape)
+
+
+def check_status(ws, stream=None) -> int:
+    """Synchronise the stream and return (and clear) the sticky device status."""
+    return lib().veda_check_status(ws.data_ptr(), _stream(stream))

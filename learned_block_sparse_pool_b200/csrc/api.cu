@@ -1,0 +1,364 @@
+// libveda host entry points: argument validation, workspace layout, launches.
+//
+// Every check here runs on the host before anything is enqueued, so an
+// invalid call returns an error code and leaves the device untouched.
+#include <math.h>
+#include <string.h>
+
+#include "veda_internal.cuh"
+
+namespace veda {
+
+int num_sms()
+{
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    return n;
+}
+
+cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s);
+bool attn_tc_supported(const AttnParams& p);
+int topk_max_tiles();
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+struct Layout {
+    int64_t nq, nr;          // query (= video key) tiles, reference tiles
+    int64_t ld_v, ld_r;      // score row strides (elements)
+    size_t qhat, khat, khat_r, sc_v, sc_r, total;
+};
+
+size_t esize(veda_dtype t) { return t == VEDA_BF16 ? 2 : 4; }
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+bool stride_ok(int64_t s, size_t es) { return s >= 0 && ((uint64_t)s * es) % 16 == 0; }
+
+veda_status check_segment(const veda_segment& s, const veda_problem& p, bool sparse, bool required)
+{
+    if (s.n_tokens < 0 || s.n_tokens > (int64_t)1 << 30) return VEDA_ERR_INVALID_ARG;
+    if (s.n_tokens == 0) {
+        if (required) return VEDA_ERR_INVALID_ARG;
+        return s.budget == 0 ? VEDA_OK : VEDA_ERR_INVALID_ARG;
+    }
+    if (!s.k || !s.v || !aligned16(s.k) || !aligned16(s.v)) return VEDA_ERR_INVALID_ARG;
+    const size_t es = esize(p.dtype);
+    if (!stride_ok(s.stride_b, es) || !stride_ok(s.stride_tok, es) || !stride_ok(s.stride_h, es))
+        return VEDA_ERR_INVALID_ARG;
+    if (s.stride_tok < p.d && s.n_tokens > 1) return VEDA_ERR_INVALID_ARG;
+    const int64_t tiles = ceil_div(s.n_tokens, p.tile);
+    if (sparse) {
+        if (s.budget < 1 || s.budget > tiles) return VEDA_ERR_INVALID_ARG;
+        if (tiles > topk_max_tiles()) return VEDA_ERR_UNSUPPORTED;
+    } else if (s.budget != 0) {
+        return VEDA_ERR_INVALID_ARG;
+    }
+    return VEDA_OK;
+}
+
+veda_status validate(const veda_problem* pp)
+{
+    if (!pp) return VEDA_ERR_INVALID_ARG;
+    const veda_problem& p = *pp;
+    if (p.B < 1 || p.H < 1 || (int64_t)p.B * p.H > 65535) return VEDA_ERR_INVALID_ARG;
+    if (p.dtype != VEDA_F32 && p.dtype != VEDA_BF16) return VEDA_ERR_INVALID_ARG;
+    if (p.d < 1 || p.tile < 1 || p.r < 1) return VEDA_ERR_INVALID_ARG;
+    if (p.d != 64 && p.d != 128) return VEDA_ERR_UNSUPPORTED;
+    if (p.tile != 64 && p.tile != 128) return VEDA_ERR_UNSUPPORTED;
+    if (p.r > 128 || p.r % 4 != 0) return VEDA_ERR_UNSUPPORTED;
+    if (!(p.softmax_scale >= 0.f) || !isfinite(p.softmax_scale)) return VEDA_ERR_INVALID_ARG;
+    if (p.flags & ~VEDA_FLAG_SIMT_ATTENTION) return VEDA_ERR_INVALID_ARG;
+    if (!p.q || !aligned16(p.q)) return VEDA_ERR_INVALID_ARG;
+    const size_t es = esize(p.dtype);
+    if (!stride_ok(p.q_stride_b, es) || !stride_ok(p.q_stride_tok, es) || !stride_ok(p.q_stride_h, es))
+        return VEDA_ERR_INVALID_ARG;
+    veda_status st;
+    if ((st = check_segment(p.video, p, true, true)) != VEDA_OK) return st;
+    if ((st = check_segment(p.ref, p, true, false)) != VEDA_OK) return st;
+    if ((st = check_segment(p.dense, p, false, false)) != VEDA_OK) return st;
+    return VEDA_OK;
+}
+
+Layout layout(const veda_problem& p)
+{
+    Layout L;
+    L.nq = ceil_div(p.video.n_tokens, p.tile);
+    L.nr = p.ref.n_tokens > 0 ? ceil_div(p.ref.n_tokens, p.tile) : 0;
+    L.ld_v = (int64_t)align_up((size_t)L.nq, 32);
+    L.ld_r = (int64_t)align_up((size_t)L.nr, 32);
+    const int64_t BH = (int64_t)p.B * p.H;
+    size_t off = kAlign;                                   // status word lives at offset 0
+    L.qhat = off;   off = align_up(off + sizeof(float) * BH * L.nq * p.r, kAlign);
+    L.khat = off;   off = align_up(off + sizeof(float) * BH * L.nq * p.r, kAlign);
+    L.khat_r = off; off = align_up(off + sizeof(float) * BH * L.nr * p.r, kAlign);
+    L.sc_v = off;   off = align_up(off + sizeof(float) * BH * L.nq * L.ld_v, kAlign);
+    L.sc_r = off;   off = align_up(off + sizeof(float) * BH * L.nq * L.ld_r, kAlign);
+    L.total = off;
+    return L;
+}
+
+veda_status check_ws(const veda_problem& p, void* ws, size_t ws_bytes, Layout* L)
+{
+    *L = layout(p);
+    if (!ws || ((uintptr_t)ws % kAlign) != 0 || ws_bytes < L->total) return VEDA_ERR_WORKSPACE;
+    return VEDA_OK;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) { return reinterpret_cast<T*>(static_cast<char*>(ws) + off); }
+
+veda_status from_cuda(cudaError_t e) { return e == cudaSuccess ? VEDA_OK : VEDA_ERR_CUDA; }
+
+Segment to_segment(const veda_segment& s, int tile)
+{
+    Segment d;
+    d.k = s.k;
+    d.v = s.v;
+    d.n = s.n_tokens;
+    d.sb = s.stride_b;
+    d.st = s.stride_tok;
+    d.sh = s.stride_h;
+    d.n_tiles = s.n_tokens > 0 ? (int32_t)ceil_div(s.n_tokens, tile) : 0;
+    d.pad = 0;
+    return d;
+}
+
+veda_status do_pool_project(const veda_problem& p, const Layout& L, const void* w_q, const void* w_k,
+                            void* ws, cudaStream_t s)
+{
+    if (!w_q || !w_k || !aligned16(w_q) || !aligned16(w_k)) return VEDA_ERR_INVALID_ARG;
+    PoolParams P;
+    memset(&P, 0, sizeof P);
+    P.B = p.B; P.H = p.H; P.d = p.d; P.T = p.tile; P.r = p.r; P.dtype = p.dtype;
+    int64_t items = 0;
+    auto add = [&](const void* x, int64_t sb, int64_t st, int64_t sh, int64_t n, const void* w, float* out) {
+        PoolJob& J = P.job[P.n_jobs++];
+        J.x = x; J.sb = sb; J.st = st; J.sh = sh; J.n_tokens = n;
+        J.n_tiles = (int32_t)ceil_div(n, p.tile);
+        J.first_item = items;
+        J.w = w; J.out = out;
+        items += (int64_t)p.B * p.H * J.n_tiles;
+    };
+    add(p.q, p.q_stride_b, p.q_stride_tok, p.q_stride_h, p.video.n_tokens, w_q, at<float>(ws, L.qhat));
+    add(p.video.k, p.video.stride_b, p.video.stride_tok, p.video.stride_h, p.video.n_tokens, w_k,
+        at<float>(ws, L.khat));
+    if (p.ref.n_tokens > 0)
+        add(p.ref.k, p.ref.stride_b, p.ref.stride_tok, p.ref.stride_h, p.ref.n_tokens, w_k,
+            at<float>(ws, L.khat_r));
+    P.total_items = items;
+    return from_cuda(launch_pool_project(P, s));
+}
+
+veda_status do_score(const veda_problem& p, const Layout& L, void* ws, cudaStream_t s)
+{
+    ScoreParams S;
+    S.qhat = at<float>(ws, L.qhat);
+    S.BH = p.B * p.H;
+    S.nq = (int32_t)L.nq;
+    S.r = p.r;
+    S.khat = at<float>(ws, L.khat);
+    S.scores = at<float>(ws, L.sc_v);
+    S.nk = (int32_t)L.nq;
+    S.ld = L.ld_v;
+    cudaError_t e = launch_score(S, s);
+    if (e == cudaSuccess && L.nr > 0) {
+        S.khat = at<float>(ws, L.khat_r);
+        S.scores = at<float>(ws, L.sc_r);
+        S.nk = (int32_t)L.nr;
+        S.ld = L.ld_r;
+        e = launch_score(S, s);
+    }
+    return from_cuda(e);
+}
+
+veda_status do_topk(const veda_problem& p, const Layout& L, int32_t* idx_v, int32_t* idx_r, void* ws,
+                    cudaStream_t s)
+{
+    if (!idx_v || (L.nr > 0) != (idx_r != nullptr)) return VEDA_ERR_INVALID_ARG;
+    TopkParams T;
+    T.status = at<uint32_t>(ws, 0);
+    T.rows = (int64_t)p.B * p.H * L.nq;
+    T.scores = at<float>(ws, L.sc_v);
+    T.ld = L.ld_v;
+    T.n = (int32_t)L.nq;
+    T.k = p.video.budget;
+    T.idx = idx_v;
+    cudaError_t e = launch_topk(T, s);
+    if (e == cudaSuccess && L.nr > 0) {
+        T.scores = at<float>(ws, L.sc_r);
+        T.ld = L.ld_r;
+        T.n = (int32_t)L.nr;
+        T.k = p.ref.budget;
+        T.idx = idx_r;
+        e = launch_topk(T, s);
+    }
+    return from_cuda(e);
+}
+
+veda_status do_attn(const veda_problem& p, const Layout& L, const int32_t* idx_v, const int32_t* idx_r,
+                    void* out, float* lse, void* ws, cudaStream_t s)
+{
+    if (!idx_v || (L.nr > 0) != (idx_r != nullptr)) return VEDA_ERR_INVALID_ARG;
+    if (!out || !aligned16(out) || (lse && ((uintptr_t)lse & 3u))) return VEDA_ERR_INVALID_ARG;
+    AttnParams A;
+    memset(&A, 0, sizeof A);
+    A.q = p.q;
+    A.qsb = p.q_stride_b; A.qst = p.q_stride_tok; A.qsh = p.q_stride_h;
+    A.video = to_segment(p.video, p.tile);
+    A.ref = to_segment(p.ref, p.tile);
+    A.dense = to_segment(p.dense, p.tile);
+    A.idx_v = idx_v;
+    A.idx_r = L.nr > 0 ? idx_r : nullptr;
+    A.k_v = p.video.budget;
+    A.k_r = L.nr > 0 ? p.ref.budget : 0;
+    A.out = out;
+    A.lse = lse;
+    A.B = p.B; A.H = p.H; A.d = p.d; A.T = p.tile; A.nq = (int32_t)L.nq;
+    A.dtype = p.dtype;
+    A.scale = p.softmax_scale > 0.f ? p.softmax_scale : 1.0f / sqrtf((float)p.d);
+    A.status = at<uint32_t>(ws, 0);
+    if (!(p.flags & VEDA_FLAG_SIMT_ATTENTION) && attn_tc_supported(A)) return from_cuda(launch_attn_tc(A, s));
+    return from_cuda(launch_attn_simt(A, s));
+}
+
+}  // namespace
+}  // namespace veda
+
+using namespace veda;
+
+extern "C" {
+
+veda_status veda_workspace_size(const veda_problem* p, size_t* bytes)
+{
+    if (!bytes) return VEDA_ERR_INVALID_ARG;
+    veda_status st = validate(p);
+    if (st != VEDA_OK) return st;
+    *bytes = layout(*p).total;
+    return VEDA_OK;
+}
+
+veda_status veda_workspace_init(void* ws, size_t ws_bytes, veda_stream_t stream)
+{
+    if (!ws || ((uintptr_t)ws % kAlign) != 0 || ws_bytes < kAlign) return VEDA_ERR_WORKSPACE;
+    return from_cuda(cudaMemsetAsync(ws, 0, kAlign, (cudaStream_t)stream));
+}
+
+veda_status veda_pool_project(const veda_problem* p, const void* w_q, const void* w_k, void* ws,
+                              size_t ws_bytes, veda_stream_t stream)
+{
+    veda_status st = validate(p);
+    if (st != VEDA_OK) return st;
+    Layout L;
+    if ((st = check_ws(*p, ws, ws_bytes, &L)) != VEDA_OK) return st;
+    return do_pool_project(*p, L, w_q, w_k, ws, (cudaStream_t)stream);
+}
+
+veda_status veda_score_tiles(const veda_problem* p, void* ws, size_t ws_bytes, veda_stream_t stream)
+{
+    veda_status st = validate(p);
+    if (st != VEDA_OK) return st;
+    Layout L;
+    if ((st = check_ws(*p, ws, ws_bytes, &L)) != VEDA_OK) return st;
+    return do_score(*p, L, ws, (cudaStream_t)stream);
+}
+
+veda_status veda_topk_tiles(const veda_problem* p, int32_t* idx_video, int32_t* idx_ref, void* ws,
+                            size_t ws_bytes, veda_stream_t stream)
+{
+    veda_status st = validate(p);
+    if (st != VEDA_OK) return st;
+    Layout L;
+    if ((st = check_ws(*p, ws, ws_bytes, &L)) != VEDA_OK) return st;
+    return do_topk(*p, L, idx_video, idx_ref, ws, (cudaStream_t)stream);
+}
+
+veda_status veda_select_tiles(const veda_problem* p, const void* w_q, const void* w_k, int32_t* idx_video,
+                              int32_t* idx_ref, void* ws, size_t ws_bytes, veda_stream_t stream)
+{
+    veda_status st = validate(p);
+    if (st != VEDA_OK) return st;
+    Layout L;
+    if ((st = check_ws(*p, ws, ws_bytes, &L)) != VEDA_OK) return st;
+    if (!idx_video || (L.nr > 0) != (idx_ref != nullptr)) return VEDA_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    if ((st = do_pool_project(*p, L, w_q, w_k, ws, s)) != VEDA_OK) return st;
+    if ((st = do_score(*p, L, ws, s)) != VEDA_OK) return st;
+    return do_topk(*p, L, idx_video, idx_ref, ws, s);
+}
+
+veda_status veda_block_sparse_attn(const veda_problem* p, const int32_t* idx_video, const int32_t* idx_ref,
+                                   void* out, float* lse, void* ws, size_t ws_bytes, veda_stream_t stream)
+{
+    veda_status st = validate(p);
+    if (st != VEDA_OK) return st;
+    if (!ws || ((uintptr_t)ws % kAlign) != 0 || ws_bytes < kAlign) return VEDA_ERR_WORKSPACE;
+    const Layout L = layout(*p);
+    return do_attn(*p, L, idx_video, idx_ref, out, lse, ws, (cudaStream_t)stream);
+}
+
+veda_status veda_attn(const veda_problem* p, const void* w_q, const void* w_k, int32_t* idx_video,
+                      int32_t* idx_ref, void* out, float* lse, void* ws, size_t ws_bytes, veda_stream_t stream)
+{
+    veda_status st = validate(p);
+    if (st != VEDA_OK) return st;
+    Layout L;
+    if ((st = check_ws(*p, ws, ws_bytes, &L)) != VEDA_OK) return st;
+    if (!idx_video || (L.nr > 0) != (idx_ref != nullptr)) return VEDA_ERR_INVALID_ARG;
+    if (!out || !aligned16(out) || (lse && ((uintptr_t)lse & 3u))) return VEDA_ERR_INVALID_ARG;
+    if (!w_q || !w_k || !aligned16(w_q) || !aligned16(w_k)) return VEDA_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    if ((st = do_pool_project(*p, L, w_q, w_k, ws, s)) != VEDA_OK) return st;
+    if ((st = do_score(*p, L, ws, s)) != VEDA_OK) return st;
+    if ((st = do_topk(*p, L, idx_video, idx_ref, ws, s)) != VEDA_OK) return st;
+    return do_attn(*p, L, idx_video, idx_ref, out, lse, ws, s);
+}
+
+veda_status veda_workspace_view(const veda_problem* p, void* ws, size_t ws_bytes, int which, const void** ptr,
+                                int64_t* ld)
+{
+    veda_status st = validate(p);
+    if (st != VEDA_OK) return st;
+    if (!ptr || !ld) return VEDA_ERR_INVALID_ARG;
+    Layout L;
+    if ((st = check_ws(*p, ws, ws_bytes, &L)) != VEDA_OK) return st;
+    const size_t offs[5] = {L.qhat, L.khat, L.khat_r, L.sc_v, L.sc_r};
+    const int64_t lds[5] = {p->r, p->r, p->r, L.ld_v, L.ld_r};
+    if (which < 0 || which > 4) return VEDA_ERR_INVALID_ARG;
+    if ((which == 2 || which == 4) && L.nr == 0) return VEDA_ERR_INVALID_ARG;
+    *ptr = static_cast<const char*>(ws) + offs[which];
+    *ld = lds[which];
+    return VEDA_OK;
+}
+
+veda_status veda_check_status(void* ws, veda_stream_t stream)
+{
+    if (!ws || ((uintptr_t)ws % kAlign) != 0) return VEDA_ERR_WORKSPACE;
+    cudaStream_t s = (cudaStream_t)stream;
+    uint32_t code = 0;
+    if (cudaMemcpyAsync(&code, ws, sizeof code, cudaMemcpyDeviceToHost, s) != cudaSuccess) return VEDA_ERR_CUDA;
+    if (cudaMemsetAsync(ws, 0, sizeof code, s) != cudaSuccess) return VEDA_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return VEDA_ERR_CUDA;
+    return code == 0 ? VEDA_OK : (veda_status)(-(int)code);
+}
+
+const char* veda_status_string(veda_status s)
+{
+    switch (s) {
+    case VEDA_OK: return "VEDA_OK";
+    case VEDA_ERR_INVALID_ARG: return "VEDA_ERR_INVALID_ARG";
+    case VEDA_ERR_UNSUPPORTED: return "VEDA_ERR_UNSUPPORTED";
+    case VEDA_ERR_WORKSPACE: return "VEDA_ERR_WORKSPACE";
+    case VEDA_ERR_CUDA: return "VEDA_ERR_CUDA";
+    case VEDA_ERR_TIMEOUT: return "VEDA_ERR_TIMEOUT";
+    case VEDA_ERR_BAD_INDEX: return "VEDA_ERR_BAD_INDEX";
+    }
+    return "VEDA_ERR_UNKNOWN";
+}
+
+}  // extern "C"

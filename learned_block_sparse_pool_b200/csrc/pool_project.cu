@@ -1,0 +1,181 @@
+// Tile pooling + selector projection (one HBM pass over Q and K).
+//
+// Computes, for every (b, h, tile i) of each job (Q with W_q; video K and
+// reference K with W_k):
+//     pooled = mean of the tokens of tile i that exist (a short last tile is
+//              averaged over its own tokens),
+//     xhat   = pooled (row vector, fp32) times W[h] ([d, r]),
+// which is the selector input: the trained query / key projections applied
+// to tile-pooled Q and K (tao.media, "Affine launches MiniMax-H3 video
+// studio...", sections "Training the Selector, Not the Generator" and "How
+// the SN120 Competition Works").
+//
+// Design (HBM-bound): a persistent grid, a multiple of the SM count, walks
+// the (job, b, h, tile) items in order; each CTA owns one contiguous run of
+// items, so it loads W[h] into shared memory once per head it meets.  Within
+// a tile, each thread owns one 16-byte column chunk of the row and a set of
+// tokens: every warp load is a 128-bit, fully coalesced access, and all of a
+// thread's loads for the tile are issued before any is consumed.
+#include <cuda_bf16.h>
+
+#include "veda_internal.cuh"
+
+namespace veda {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kMaxTile = 128;
+
+__device__ __forceinline__ void unpack(const uint4& raw, float* f, const float*)
+{
+    f[0] = __uint_as_float(raw.x);
+    f[1] = __uint_as_float(raw.y);
+    f[2] = __uint_as_float(raw.z);
+    f[3] = __uint_as_float(raw.w);
+}
+
+__device__ __forceinline__ void unpack(const uint4& raw, float* f, const __nv_bfloat16*)
+{
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+__device__ __forceinline__ uint4 load_stream(const void* p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+template <typename Tin, int D>
+__global__ void __launch_bounds__(kThreads) pool_project_kernel(const PoolParams P)
+{
+    constexpr int EPC = 16 / sizeof(Tin);      // elements per 16-byte chunk
+    constexpr int CPR = D / EPC;               // chunks per token row
+    constexpr int RP = kThreads / CPR;         // token rows loaded in parallel
+    constexpr int LOADS = kMaxTile / RP;       // loads per thread per tile (max)
+
+    extern __shared__ float smem[];
+    const int r = P.r;
+    float* w_s = smem;                         // [D][r]
+    float* part = w_s + D * r;                 // [RP][D]
+    float* pooled = part + RP * D;             // [D]
+    float* proj = pooled + D;                  // [groups][r]
+
+    const int tid = threadIdx.x;
+    const int chunk = tid % CPR;
+    const int row0 = tid / CPR;
+    const int groups = kThreads / r;
+
+    const int64_t it0 = (int64_t)blockIdx.x * P.total_items / gridDim.x;
+    const int64_t it1 = (int64_t)(blockIdx.x + 1) * P.total_items / gridDim.x;
+    int cur_job = -1, cur_h = -1;
+
+    for (int64_t it = it0; it < it1; ++it) {
+        int j = 0;
+        while (j + 1 < P.n_jobs && it >= P.job[j + 1].first_item) ++j;
+        const PoolJob& J = P.job[j];
+        const int64_t local = it - J.first_item;
+        const int i = (int)(local % J.n_tiles);
+        const int64_t bh = local / J.n_tiles;
+        const int h = (int)(bh % P.H);
+        const int b = (int)(bh / P.H);
+
+        if (j != cur_job || h != cur_h) {
+            __syncthreads();   // the previous item's projection no longer reads w_s
+            const Tin* W = static_cast<const Tin*>(J.w) + (int64_t)h * D * r;
+            for (int e = tid; e < D * r; e += kThreads) w_s[e] = to_f32(W[e]);
+            cur_job = j;
+            cur_h = h;
+        }
+
+        // ---- pool: sum this thread's tokens of its 16-byte column chunk ----
+        const int64_t t0 = (int64_t)i * P.T;
+        const int64_t t1 = min(J.n_tokens, t0 + P.T);
+        const Tin* base = static_cast<const Tin*>(J.x) + (int64_t)b * J.sb + (int64_t)h * J.sh +
+                          (int64_t)chunk * EPC;
+        uint4 raw[LOADS];
+#pragma unroll
+        for (int u = 0; u < LOADS; ++u) {
+            const int64_t t = t0 + row0 + (int64_t)u * RP;
+            raw[u] = (t < t1) ? load_stream(base + t * J.st) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        float acc[EPC];
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
+#pragma unroll
+        for (int u = 0; u < LOADS; ++u) {
+            float f[EPC];
+            unpack(raw[u], f, (const Tin*)nullptr);
+#pragma unroll
+            for (int e = 0; e < EPC; ++e) acc[e] += f[e];
+        }
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) part[row0 * D + chunk * EPC + e] = acc[e];
+        __syncthreads();
+        if (tid < D) {
+            float s = 0.f;
+#pragma unroll 8
+            for (int q = 0; q < RP; ++q) s += part[q * D + tid];
+            pooled[tid] = s / (float)(t1 - t0);
+        }
+        __syncthreads();
+
+        // ---- project: xhat[c] = sum_e pooled[e] * W[h][e][c] ----
+        const int c = tid % r;
+        const int g = tid / r;
+        if (g < groups) {
+            float s = 0.f;
+            for (int e = g; e < D; e += groups) s += pooled[e] * w_s[e * r + c];
+            proj[g * r + c] = s;
+        }
+        __syncthreads();
+        if (tid < r) {
+            float s = 0.f;
+            for (int q = 0; q < groups; ++q) s += proj[q * r + tid];
+            J.out[((int64_t)(b * P.H + h) * J.n_tiles + i) * r + tid] = s;
+        }
+    }
+}
+
+template <typename Tin, int D>
+cudaError_t launch_typed(const PoolParams& p, cudaStream_t s)
+{
+    constexpr int EPC = 16 / sizeof(Tin);
+    constexpr int RP = kThreads / (D / EPC);
+    const int groups = kThreads / p.r;
+    const size_t smem = sizeof(float) * ((size_t)D * p.r + RP * D + D + (size_t)groups * p.r);
+    auto kern = pool_project_kernel<Tin, D>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) per_sm = 1;
+    int64_t grid = (int64_t)num_sms() * per_sm;
+    if (grid > p.total_items) grid = p.total_items;
+    kern<<<(unsigned)grid, kThreads, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_pool_project(const PoolParams& p, cudaStream_t s)
+{
+    if (p.total_items == 0) return cudaSuccess;
+    if (p.dtype == VEDA_BF16) {
+        return p.d == 128 ? launch_typed<__nv_bfloat16, 128>(p, s) : launch_typed<__nv_bfloat16, 64>(p, s);
+    }
+    return p.d == 128 ? launch_typed<float, 128>(p, s) : launch_typed<float, 64>(p, s);
+}
+
+}  // namespace veda

@@ -1,0 +1,93 @@
+// Internal declarations of libveda (not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "veda.h"
+
+namespace veda {
+
+// Device-side status codes are stored as the positive value of the
+// veda_status they map to (0 = no error); the first error sticks.
+__device__ __forceinline__ void record_status(uint32_t* status, veda_status s)
+{
+    if (status) atomicCAS(status, 0u, (uint32_t)(-(int)s));
+}
+
+struct Segment {            // one key/value segment as device code sees it
+    const void* k;
+    const void* v;
+    int64_t n;              // tokens
+    int64_t sb, st, sh;     // element strides
+    int32_t n_tiles;
+    int32_t pad;
+};
+
+// ---- tile pooling + selector projection --------------------------------
+struct PoolJob {
+    const void* x;          // [B, n, H, d]
+    int64_t sb, st, sh;
+    int64_t n_tokens;
+    int64_t first_item;     // items before this job (item = (b, h, tile))
+    const void* w;          // [H, d, r]
+    float* out;             // [B, H, n_tiles, r]
+    int32_t n_tiles;
+    int32_t pad;
+};
+
+struct PoolParams {
+    PoolJob job[3];
+    int32_t n_jobs;
+    int32_t B, H, d, T, r;
+    int32_t dtype;
+    int64_t total_items;
+};
+
+cudaError_t launch_pool_project(const PoolParams& p, cudaStream_t s);
+
+// ---- tile scores ----------------------------------------------------------
+struct ScoreParams {
+    const float* qhat;      // [BH, nq, r]
+    const float* khat;      // [BH, nk, r]
+    float* scores;          // [BH, nq, ld]
+    int32_t BH, nq, nk, r;
+    int64_t ld;
+};
+
+cudaError_t launch_score(const ScoreParams& p, cudaStream_t s);
+
+// ---- fixed-budget top-k -------------------------------------------------
+struct TopkParams {
+    const float* scores;    // [rows, ld]
+    int64_t ld;
+    int64_t rows;
+    int32_t n;              // key tiles per row
+    int32_t k;              // budget
+    int32_t* idx;           // [rows, k]
+    uint32_t* status;
+};
+
+cudaError_t launch_topk(const TopkParams& p, cudaStream_t s);
+
+// ---- attention ----------------------------------------------------------
+struct AttnParams {
+    const void* q;
+    int64_t qsb, qst, qsh;
+    Segment video, ref, dense;
+    const int32_t* idx_v;   // [B, H, nq, k_v]
+    const int32_t* idx_r;   // [B, H, nq, k_r] or null
+    int32_t k_v, k_r;
+    void* out;              // [B, n_video, H, d]
+    float* lse;             // [B, H, n_video] or null
+    int32_t B, H, d, T, nq;
+    int32_t dtype;
+    float scale;            // softmax scale (natural-log units)
+    uint32_t* status;
+};
+
+cudaError_t launch_attn_simt(const AttnParams& p, cudaStream_t s);
+
+int num_sms();
+
+}  // namespace veda

@@ -1,0 +1,96 @@
+"""Comparison helpers for GPU-vs-oracle parity tests.
+
+Tolerances (stated once, used by every parity test):
+  * selection: kept-tile sets bit-exact, except rows whose differing tiles all
+    score within TIE_REL (relative, in the oracle's fp64) of the row's k-th
+    score -- a near-tie the fp32 kernels may legitimately order either way;
+    every such row is reported.
+  * attention, fp32 problems: max-abs <= 1e-4 and relative L2 <= 1e-4.
+  * attention, bf16 problems: max-abs <= 2e-2 and relative L2 <= 5e-3
+    (the output itself is rounded to bf16, 2^-9 relative).
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+from typing import List
+
+import numpy as np
+import torch
+
+TIE_REL = 1e-4
+TOL = {torch.float32: (1e-4, 1e-4), torch.bfloat16: (2e-2, 5e-3)}
+
+
+@dataclass
+class SelectionReport:
+    rows: int
+    mismatched: int = 0
+    tie_band: List[int] = field(default_factory=list)
+    violations: List[int] = field(default_factory=list)
+
+
+def compare_selection(oracle_mod, gpu_idx: np.ndarray, ref_idx: np.ndarray, kth: np.ndarray,
+                      qhat: np.ndarray, khat: np.ndarray) -> SelectionReport:
+    g = gpu_idx.reshape(-1, gpu_idx.shape[-1])
+    o = ref_idx.reshape(-1, ref_idx.shape[-1])
+    rep = SelectionReport(rows=g.shape[0])
+    bad = np.nonzero((g != o).any(axis=1))[0]
+    rep.mismatched = len(bad)
+    if len(bad) == 0:
+        return rep
+    s = oracle_mod.scores(qhat, khat, bad)
+    kth_flat = kth.reshape(-1)
+    for q, row in enumerate(bad):
+        diff = set(g[row].tolist()) ^ set(o[row].tolist())
+        if len(set(g[row].tolist())) != g.shape[1] or any(j < 0 or j >= s.shape[1] for j in diff):
+            rep.violations.append(int(row))
+            continue
+        sk = kth_flat[row]
+        ok = all(abs(s[q, j] - sk) <= TIE_REL * max(abs(s[q, j]), abs(sk)) for j in diff)
+        (rep.tie_band if ok else rep.violations).append(int(row))
+    return rep
+
+
+def assert_selection(rep: SelectionReport, what: str = ""):
+    assert not rep.violations, (f"{what}: {len(rep.violations)} rows differ outside the tie band "
+                                f"(first {rep.violations[:5]})")
+    if rep.tie_band:
+        print(f"[tie band] {what}: {len(rep.tie_band)} of {rep.rows} rows differ only inside the "
+              f"{TIE_REL:g} relative tie band: {rep.tie_band[:10]}")
+
+
+def errors(got: np.ndarray, want: np.ndarray):
+    m = ~np.isnan(want)
+    d = got[m] - want[m]
+    max_abs = float(np.abs(d).max()) if d.size else 0.0
+    rel_l2 = float(np.linalg.norm(d) / max(np.linalg.norm(want[m]), 1e-30)) if d.size else 0.0
+    return max_abs, rel_l2
+
+
+def assert_close(got: np.ndarray, want: np.ndarray, dtype, what: str = ""):
+    tol_abs, tol_rel = TOL[dtype]
+    max_abs, rel_l2 = errors(got, want)
+    assert np.isfinite(got[~np.isnan(want)]).all(), f"{what}: non-finite output"
+    assert max_abs <= tol_abs and rel_l2 <= tol_rel, \
+        f"{what}: max-abs {max_abs:.3g} (<= {tol_abs}), rel-L2 {rel_l2:.3g} (<= {tol_rel})"
+    return max_abs, rel_l2
+
+
+def gather_units(out: torch.Tensor, units, T: int) -> np.ndarray:
+    """GPU output [B, N, H, d] -> [n_units, T, d] fp64 (NaN past the end)."""
+    B, N, H, d = out.shape
+    res = np.full((len(units), T, d), np.nan)
+    host = {}
+    for u, (b, h, i) in enumerate(units):
+        t0, t1 = i * T, min(N, (i + 1) * T)
+        res[u, :t1 - t0] = out[b, t0:t1, h].float().cpu().double().numpy()
+    return res
+
+
+def gather_lse(lse: torch.Tensor, units, T: int) -> np.ndarray:
+    B, H, N = lse.shape
+    res = np.full((len(units), T), np.nan)
+    for u, (b, h, i) in enumerate(units):
+        t0, t1 = i * T, min(N, (i + 1) * T)
+        res[u, :t1 - t0] = lse[b, h, t0:t1].cpu().double().numpy()
+    return res

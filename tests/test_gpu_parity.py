@@ -1,0 +1,265 @@
+"""GPU parity: the CUDA library (through its C ABI) against the CPU oracle,
+element by element, on seeded synthetic inputs.
+
+  * selection (veda_select_tiles): kept-tile sets bit-exact against the
+    oracle's, except reported near-ties (tests/parity.py);
+  * pooled projections: fp32 workspace values against the oracle's fp64;
+  * attention (veda_block_sparse_attn) on the ORACLE's kept tiles, so both
+    sides attend to the same keys, within the fp32 / bf16 tolerances;
+  * the fused veda_attn against the two-step path.
+Sizes: the tiny workload in full; reduced workloads spanning several tiles
+with ragged video / reference / dense tails; edge cases (budget = every
+tile, budget 1, batch 2 with non-packed strides, an out-of-range index);
+and every full-size workload with selection checked on all rows and
+attention on a seeded sample of (b, h, query tile) units.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import learned_block_sparse_pool_b200 as veda
+import workloads
+from parity import assert_close, assert_selection, compare_selection, gather_lse, gather_units
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from learned_block_sparse_pool_b200 import build
+    build.build()
+    return torch.device("cuda:0")
+
+
+def to_dev(inp, dev):
+    return {k: v.to(dev) for k, v in inp.items()}
+
+
+def make_problem(w, g, flags=0, budget=None):
+    return veda.Problem(g["q"], g["k"], g["v"], tile=w.T, r=w.r,
+                        budget=w.budget_video if budget is None else budget,
+                        k_ref=g.get("k_ref"), v_ref=g.get("v_ref"),
+                        budget_ref=w.budget_ref if "k_ref" in g else 0,
+                        k_dense=g.get("k_dense"), v_dense=g.get("v_dense"), flags=flags)
+
+
+def gpu_select(p, g, ws):
+    iv, ir = veda.alloc_indices(p)
+    veda.select_tiles(p, g["w_q"], g["w_k"], iv, ir, ws)
+    return iv, ir
+
+
+def check_selection(oracle_mod, p, ws, iv, ir, sel, what):
+    r = p.c.r
+    qh = veda.workspace_view(p, ws, 0)[..., :r].double().cpu().numpy()
+    kh = veda.workspace_view(p, ws, 1)[..., :r].double().cpu().numpy()
+    np.testing.assert_allclose(qh, sel["qhat"], rtol=2e-5, atol=2e-6)
+    np.testing.assert_allclose(kh, sel["khat"], rtol=2e-5, atol=2e-6)
+    rep = compare_selection(oracle_mod, iv.cpu().numpy(), sel["idx_v"], sel["kth_v"], sel["qhat"], sel["khat"])
+    assert_selection(rep, what + " video")
+    if ir is not None:
+        rep_r = compare_selection(oracle_mod, ir.cpu().numpy(), sel["idx_r"], sel["kth_r"], sel["qhat"],
+                                  sel["khat_r"])
+        assert_selection(rep_r, what + " reference")
+    return rep
+
+
+def check_attention(oracle_mod, w, inp, p, ws, sel, units, what, with_lse=True):
+    g_iv = torch.from_numpy(sel["idx_v"]).to(p.device)
+    g_ir = torch.from_numpy(sel["idx_r"]).to(p.device) if "idx_r" in sel else None
+    out, lse = veda.alloc_output(p, with_lse=with_lse)
+    out.fill_(float("nan"))
+    veda.block_sparse_attn(p, g_iv, g_ir, out, lse, ws)
+    assert veda.check_status(ws) == 0
+    want, want_lse = oracle_mod.attend_units(inp, w.T, sel["idx_v"], sel.get("idx_r"), units)
+    got = gather_units(out, units, w.T)
+    err = assert_close(got, want, p.dtype, what)
+    if with_lse:
+        got_lse = gather_lse(lse, units, w.T)
+        m = ~np.isnan(want_lse)
+        assert np.abs(got_lse[m] - want_lse[m]).max() < (1e-4 if p.dtype == torch.float32 else 2e-2)
+    return out, err
+
+
+# ---------------------------------------------------------------------------
+# tiny workload (fp32), in full
+# ---------------------------------------------------------------------------
+
+def test_tiny_workload(dev, oracle_mod):
+    w = workloads.get("tiny")
+    inp = workloads.make_inputs(w)
+    g = to_dev(inp, dev)
+    p = make_problem(w, g)
+    ws = veda.workspace(p)
+    iv, ir = gpu_select(p, g, ws)
+    sel = oracle_mod.select_tiles(inp, w.T, w.budget_video)
+    check_selection(oracle_mod, p, ws, iv, ir, sel, "tiny")
+    units = [(0, h, i) for h in range(w.H) for i in range(w.n_q_tiles)]
+    out, err = check_attention(oracle_mod, w, inp, p, ws, sel, units, "tiny attention")
+    print(f"tiny: max-abs {err[0]:.3g} rel-L2 {err[1]:.3g}")
+
+    # fused call: same kept tiles as veda_select_tiles and the same output bits
+    iv2, ir2 = veda.alloc_indices(p)
+    out2, _ = veda.alloc_output(p)
+    veda.attn(p, g["w_q"], g["w_k"], iv2, ir2, out2, None, ws)
+    assert veda.check_status(ws) == 0
+    assert torch.equal(iv2, iv)
+    out3, _ = veda.alloc_output(p)
+    veda.block_sparse_attn(p, iv, None, out3, None, ws)
+    assert torch.equal(out2, out3)
+
+
+def test_tiny_full_budget_is_dense(dev, oracle_mod):
+    w = workloads.get("tiny").with_budget(64)
+    inp = workloads.make_inputs(w)
+    g = to_dev(inp, dev)
+    p = make_problem(w, g)
+    ws = veda.workspace(p)
+    iv, _ = gpu_select(p, g, ws)
+    assert (iv.cpu().numpy() == np.arange(64)).all()
+    sel = {"idx_v": iv.cpu().numpy()}
+    units = [(0, h, i) for h in range(w.H) for i in (0, 1, 31, 62, 63)]
+    check_attention(oracle_mod, w, inp, p, ws, sel, units, "tiny dense")
+
+
+# ---------------------------------------------------------------------------
+# reduced workloads: several tiles, ragged tails, reference segment
+# ---------------------------------------------------------------------------
+
+def _reduced(name, **kw):
+    base = dict(frames=3, Y=16, X=21, H=4, dense=(("text", 200),), budget_video=3)
+    base.update(kw)
+    return workloads.small(name, **base)
+
+
+REDUCED = {
+    "t2v_ragged": lambda: _reduced("t2v_5.17s"),
+    "r2va_ragged": lambda: _reduced("r2va_5.17s", ref_frames=1, budget_ref=2,
+                                    dense=(("text", 130), ("vlm", 70), ("audio", 64))),
+    "portrait_boost": lambda: _reduced("portrait_10.13s", frames=5, Y=21, X=16, budget_video=4),
+    "t2v_no_dense": lambda: _reduced("t2v_5.17s", dense=(), budget_video=2),
+    "fp32_d128": lambda: _reduced("t2v_5.17s", dtype="f32"),
+    "bf16_d64_t64": lambda: _reduced("t2v_5.17s", d=64, T=64, r=32, budget_video=5),
+}
+
+
+@pytest.mark.parametrize("simt", [False, True], ids=["default", "simt"])
+@pytest.mark.parametrize("name", sorted(REDUCED))
+def test_reduced_workloads(dev, oracle_mod, name, simt):
+    w = REDUCED[name]()
+    inp = workloads.make_inputs(w)
+    g = to_dev(inp, dev)
+    p = make_problem(w, g, flags=veda.binding.VEDA_FLAG_SIMT_ATTENTION if simt else 0)
+    ws = veda.workspace(p)
+    iv, ir = gpu_select(p, g, ws)
+    sel = oracle_mod.select_tiles(inp, w.T, w.budget_video, w.budget_ref if w.ref_frames else 0)
+    check_selection(oracle_mod, p, ws, iv, ir, sel, name)
+    units = [(0, h, i) for h in range(w.H) for i in range(w.n_q_tiles)]
+    check_attention(oracle_mod, w, inp, p, ws, sel, units, name)
+
+
+# ---------------------------------------------------------------------------
+# edge cases
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_budget_every_tile_and_budget_one(dev, oracle_mod, dtype):
+    w = _reduced("t2v_5.17s", dtype=dtype)
+    inp = workloads.make_inputs(w)
+    g = to_dev(inp, dev)
+    n = w.n_q_tiles
+    for k in (n, 1):
+        wk = w.with_budget(k)
+        p = make_problem(wk, g)
+        ws = veda.workspace(p)
+        iv, ir = gpu_select(p, g, ws)
+        sel = oracle_mod.select_tiles(inp, w.T, k)
+        check_selection(oracle_mod, p, ws, iv, ir, sel, f"budget {k}")
+        units = [(0, h, i) for h in range(w.H) for i in range(n)]
+        check_attention(oracle_mod, wk, inp, p, ws, sel, units, f"budget {k}")
+
+
+def test_batch_two_non_packed_strides(dev, oracle_mod):
+    """B = 2; q/k/v stored [B, H, N, d] and passed as [B, N, H, d] views."""
+    w = _reduced("r2va_5.17s", B=2, ref_frames=1, budget_ref=2)
+    inp = workloads.make_inputs(w)
+    inp = {k: (v.permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3) if v.dim() == 4 else v)
+           for k, v in inp.items()}
+    g = {k: (v.permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3).to(dev) if v.dim() == 4 else v.to(dev))
+         for k, v in inp.items()}
+    assert not g["q"].is_contiguous() and g["q"].stride(2) == g["q"].shape[1] * g["q"].shape[3]
+    p = make_problem(w, g)
+    ws = veda.workspace(p)
+    iv, ir = gpu_select(p, g, ws)
+    sel = oracle_mod.select_tiles(inp, w.T, w.budget_video, w.budget_ref)
+    check_selection(oracle_mod, p, ws, iv, ir, sel, "batch2")
+    units = [(b, h, i) for b in range(2) for h in range(w.H) for i in range(w.n_q_tiles)]
+    check_attention(oracle_mod, w, inp, p, ws, sel, units, "batch2")
+
+
+@pytest.mark.parametrize("simt", [False, True], ids=["default", "simt"])
+def test_out_of_range_index_is_flagged(dev, simt):
+    w = _reduced("t2v_5.17s")
+    g = to_dev(workloads.make_inputs(w), dev)
+    p = make_problem(w, g, flags=veda.binding.VEDA_FLAG_SIMT_ATTENTION if simt else 0)
+    ws = veda.workspace(p)
+    iv, _ = gpu_select(p, g, ws)
+    assert veda.check_status(ws) == 0
+    bad = iv.clone()
+    bad[0, 1, 2, 0] = w.n_q_tiles + 5
+    out, _ = veda.alloc_output(p)
+    veda.block_sparse_attn(p, bad, None, out, None, ws)
+    assert veda.check_status(ws) == veda.binding.VEDA_ERR_BAD_INDEX
+    assert veda.check_status(ws) == 0            # reading re-arms the status word
+
+
+def test_simt_and_default_paths_agree(dev):
+    w = _reduced("r2va_5.17s", ref_frames=1, budget_ref=2)
+    g = to_dev(workloads.make_inputs(w), dev)
+    outs = []
+    for flags in (0, veda.binding.VEDA_FLAG_SIMT_ATTENTION):
+        p = make_problem(w, g, flags=flags)
+        ws = veda.workspace(p)
+        iv, ir = gpu_select(p, g, ws)
+        out, _ = veda.alloc_output(p)
+        veda.block_sparse_attn(p, iv, ir, out, None, ws)
+        assert veda.check_status(ws) == 0
+        outs.append(out.float())
+    d = (outs[0] - outs[1]).abs().max().item()
+    assert d <= 2e-2, d
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads: every selection row, a sample of attention units
+# ---------------------------------------------------------------------------
+
+FULL = ["t2v_5.17s", "t2v_14.38s", "r2va_5.17s", "portrait_10.13s"]
+
+
+def sample_units(w, n_units=64, seed=0):
+    rng = np.random.default_rng(seed)
+    units = {(0, 0, 0), (0, w.H - 1, w.n_q_tiles - 1), (0, w.H // 2, w.n_q_tiles - 1), (0, 1, 0)}
+    while len(units) < n_units:
+        units.add((0, int(rng.integers(w.H)), int(rng.integers(w.n_q_tiles))))
+    return sorted(units)
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_workload(dev, oracle_mod, name):
+    w = workloads.get(name)
+    g = workloads.make_inputs(w, device=dev)
+    p = make_problem(w, g)
+    ws = veda.workspace(p)
+    iv, ir = gpu_select(p, g, ws)
+    torch.cuda.synchronize()
+    host = {k: v.cpu() for k, v in g.items()}
+    sel = oracle_mod.select_tiles(host, w.T, w.budget_video, w.budget_ref if w.ref_frames else 0)
+    rep = check_selection(oracle_mod, p, ws, iv, ir, sel, name)
+    print(f"{name}: {rep.rows} selection rows, {len(rep.tie_band)} inside the tie band")
+    units = sample_units(w)
+    _, err = check_attention(oracle_mod, w, host, p, ws, sel, units, name)
+    print(f"{name}: attention on {len(units)} units: max-abs {err[0]:.3g} rel-L2 {err[1]:.3g}")
