@@ -160,6 +160,28 @@ VEDA_API veda_status veda_score_tiles(const veda_problem* p, void* ws, size_t ws
 VEDA_API veda_status veda_topk_tiles(const veda_problem* p, int32_t* idx_video, int32_t* idx_ref,
                             void* ws, size_t ws_bytes, veda_stream_t stream);
 
+/* Tile selection without a workspace, for callers that cannot allocate
+ * device memory when they call: a serving engine that plans all memory up
+ * front and forbids allocation once requests flow, a plugin whose enqueue
+ * hook may not allocate, or a latency-critical loop that cannot afford the
+ * device synchronisation cudaMalloc implies.  The pages have no counterpart
+ * of this call; it exists only for such callers.
+ *   Computes exactly what veda_select_tiles() computes (same kernels), with
+ *   its scratch in a 64 MiB array that this library reserves statically on
+ *   every GPU that uses it and keeps until the process exits.  The problem is
+ *   processed one batch entry and one group of heads at a time; a problem
+ *   where the scores of a single head do not fit (about 4000 key tiles at
+ *   r = 64) returns VEDA_ERR_WORKSPACE without launching anything.
+ *   The call allocates nothing.  Its first call on each device looks up the
+ *   array's device address (cudaGetSymbolAddress), so make that first call
+ *   before capturing the stream into a CUDA graph.  All calls share the one
+ *   array, which keeps the last call's contents: calls that can overlap on
+ *   the GPU (different streams without ordering) race with each other;
+ *   calls on one stream are ordered and safe.
+ *   Arguments as for veda_select_tiles(), without ws / ws_bytes. */
+VEDA_API veda_status veda_select_tiles_noalloc(const veda_problem* p, const void* w_q, const void* w_k,
+                                               int32_t* idx_video, int32_t* idx_ref, veda_stream_t stream);
+
 /* Read-only views of the workspace (device pointers), for tests:
  *   which = 0: qhat [B,H,n_q_tiles,r] fp32     1: khat video [B,H,n_q_tiles,r]
  *           2: khat ref [B,H,n_ref_tiles,r]    3: scores video [B,H,n_q_tiles,ld]

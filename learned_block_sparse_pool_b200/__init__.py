@@ -9,8 +9,8 @@ ctypes marshalling layer over it.  Build the library with
 """
 from .binding import (EXPORTS, LIB_PATH, Problem, VedaError, alloc_indices, alloc_output, attn,
                       block_sparse_attn, check_status, lib, pool_project, score_tiles, select_tiles,
-                      status_string, topk_tiles, workspace, workspace_size, workspace_view)
+                      select_tiles_noalloc, status_string, topk_tiles, workspace, workspace_size, workspace_view)
 
 __all__ = ["EXPORTS", "LIB_PATH", "Problem", "VedaError", "alloc_indices", "alloc_output", "attn",
            "block_sparse_attn", "check_status", "lib", "pool_project", "score_tiles", "select_tiles",
-           "status_string", "topk_tiles", "workspace", "workspace_size", "workspace_view"]
+           "select_tiles_noalloc", "status_string", "topk_tiles", "workspace", "workspace_size", "workspace_view"]

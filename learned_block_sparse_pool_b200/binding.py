@@ -28,7 +28,7 @@ VEDA_FLAG_SIMT_ATTENTION = 1
 
 EXPORTS = ("veda_workspace_size", "veda_workspace_init", "veda_select_tiles", "veda_block_sparse_attn",
            "veda_attn", "veda_pool_project", "veda_score_tiles", "veda_topk_tiles", "veda_workspace_view",
-           "veda_check_status", "veda_status_string")
+           "veda_check_status", "veda_status_string", "veda_select_tiles_noalloc")
 
 
 class VedaError(RuntimeError):
@@ -75,6 +75,7 @@ def lib() -> ctypes.CDLL:
         L.veda_workspace_view.argtypes = [P, vp, sz, ctypes.c_int, ctypes.POINTER(ctypes.c_void_p),
                                           ctypes.POINTER(ctypes.c_int64)]
         L.veda_check_status.argtypes = [vp, vp]
+        L.veda_select_tiles_noalloc.argtypes = [P, vp, vp, i32p, i32p, vp]
         L.veda_status_string.argtypes = [ctypes.c_int]
         L.veda_status_string.restype = ctypes.c_char_p
         for name in EXPORTS:
@@ -190,6 +191,13 @@ def alloc_output(p: Problem, with_lse: bool = False):
 def select_tiles(p: Problem, w_q, w_k, idx_v, idx_r, ws, stream=None) -> None:
     _check(lib().veda_select_tiles(p.ref(), w_q.data_ptr(), w_k.data_ptr(), _ptr(idx_v), _ptr(idx_r),
                                    ws.data_ptr(), ws.numel(), _stream(stream)), "veda_select_tiles")
+
+
+def select_tiles_noalloc(p: Problem, w_q, w_k, idx_v, idx_r, stream=None) -> None:
+    """veda_select_tiles without a workspace: scratch lives in a static
+    per-device array inside the library (see include/veda.h)."""
+    _check(lib().veda_select_tiles_noalloc(p.ref(), w_q.data_ptr(), w_k.data_ptr(), _ptr(idx_v), _ptr(idx_r),
+                                           _stream(stream)), "veda_select_tiles_noalloc")
 
 
 def block_sparse_attn(p: Problem, idx_v, idx_r, out, lse, ws, stream=None) -> None:

@@ -1,0 +1,84 @@
+"""veda_select_tiles_noalloc: tile selection for callers that cannot
+allocate device memory at call time (a serving engine with a pre-planned
+memory pool, a plugin enqueue hook that must not allocate, a loop that cannot
+take cudaMalloc's device synchronisation).  Its scratch is a static per-device
+array inside the library, so the caller passes only inputs and outputs.
+
+Checked through the C ABI against veda_select_tiles (the workspace entry
+point): the kept tiles must be identical, on two calls in a row (the static
+array keeps the previous call's contents, which must not leak into the next
+result).  This file is collected last on purpose.
+"""
+import ctypes
+
+import pytest
+import torch
+
+import learned_block_sparse_pool_b200 as veda
+import workloads
+from learned_block_sparse_pool_b200 import binding as B
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from learned_block_sparse_pool_b200 import build
+    build.build()
+    return torch.device("cuda:0")
+
+
+def _problem(w, g):
+    return veda.Problem(g["q"], g["k"], g["v"], tile=w.T, r=w.r, budget=w.budget_video,
+                        k_ref=g.get("k_ref"), v_ref=g.get("v_ref"),
+                        budget_ref=w.budget_ref if "k_ref" in g else 0,
+                        k_dense=g.get("k_dense"), v_dense=g.get("v_dense"))
+
+
+def _compare_two_calls(w, g):
+    p = _problem(w, g)
+    ws = veda.workspace(p)
+    iv, ir = veda.alloc_indices(p)
+    veda.select_tiles(p, g["w_q"], g["w_k"], iv, ir, ws)
+    assert veda.check_status(ws) == 0
+    for call in range(2):
+        jv, jr = veda.alloc_indices(p)
+        jv.fill_(-7)
+        if jr is not None:
+            jr.fill_(-7)
+        veda.select_tiles_noalloc(p, g["w_q"], g["w_k"], jv, jr)
+        torch.cuda.synchronize()
+        assert torch.equal(jv, iv), f"call {call}: video tiles differ"
+        if ir is not None:
+            assert torch.equal(jr, ir), f"call {call}: reference tiles differ"
+
+
+def test_noalloc_matches_workspace_entry_full_clip(dev):
+    """5.17 s clip (32 heads, 977 tiles): the static array holds 14 heads'
+    scores, so the call runs in three head groups."""
+    w = workloads.get("t2v_5.17s")
+    _compare_two_calls(w, workloads.make_inputs(w, device=dev))
+
+
+def test_noalloc_matches_workspace_entry_batch_and_reference(dev):
+    w = workloads.small("r2va_5.17s", B=2, frames=3, Y=16, X=21, H=4, ref_frames=1, budget_video=3,
+                        budget_ref=2, dense=(("text", 200),))
+    _compare_two_calls(w, {k: v.to(dev) for k, v in workloads.make_inputs(w).items()})
+
+
+def test_noalloc_rejects_a_head_that_does_not_fit(dev):
+    """4096 key tiles: one head's scores alone exceed the static array."""
+    p = B.veda_problem()
+    p.B, p.H, p.d, p.tile, p.r = 1, 1, 128, 128, 64
+    p.dtype = B.VEDA_BF16
+    n = 4096 * 128
+    p.q = 0x100000
+    p.q_stride_b, p.q_stride_tok, p.q_stride_h = n * 128, 128, 128
+    p.video.k, p.video.v = 0x200000, 0x300000
+    p.video.n_tokens = n
+    p.video.stride_b, p.video.stride_tok, p.video.stride_h = n * 128, 128, 128
+    p.video.budget = 8
+    st = veda.lib().veda_select_tiles_noalloc(ctypes.byref(p), 0x400000, 0x500000, 0x600000, None, None)
+    assert st == B.VEDA_ERR_WORKSPACE
