@@ -45,6 +45,7 @@ def parse():
     ap.add_argument("--impl", choices=["veda", "reference"], default="veda")
     ap.add_argument("--workload", default="t2v_5.17s", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--budget", type=int, default=0, help="override the video budget")
+    ap.add_argument("--heads", type=int, default=0, help="override the head count (smaller profiling cases)")
     ap.add_argument("--simt", action="store_true", help="use the SIMT attention kernel")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -176,6 +177,8 @@ def main():
     w = workloads.get(args.workload)
     if args.budget:
         w = w.with_budget(args.budget)
+    if args.heads:
+        w = workloads.small(w.name, H=args.heads, budget_video=w.budget_video)
     n = world
 
     if args.impl == "reference":

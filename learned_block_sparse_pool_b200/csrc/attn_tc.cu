@@ -226,6 +226,40 @@ __device__ __forceinline__ float fast_exp2(float x)
     return y;
 }
 
+__device__ __forceinline__ float max3f(float a, float b, float c)
+{
+    float m;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(a), "f"(b), "f"(c));
+    return m;
+}
+
+// Packed pairs of fp32 (two lanes of one 64-bit register) for the f32x2 ops.
+__device__ __forceinline__ uint64_t pk2(uint32_t lo, uint32_t hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+    return r;
+}
+
+__device__ __forceinline__ void upk2(uint64_t v, float& lo, float& hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle, sm100 format (version 1).
 __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo)
 {
@@ -418,6 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             const int h = (int)(bh % P.H), b = (int)(bh / P.H);
             float m_run = -INFINITY, l = 0.f;
             for (int j = 0; j < n_list; ++j, ++t) {
+                const TileRef r = resolve(P, u, j);      // index load overlaps the wait below
                 const uint32_t sb = t & 1;
                 if (!(ok = warp_wait(sm, &sm.s_full[sb], (t >> 1) & 1, P.status))) break;
                 tc_fence_after();
@@ -431,14 +466,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 tc_fence_before();
                 mbar_arrive(&sm.s_free[sb]);
 
-                const TileRef r = resolve(P, u, j);
-                if (r.valid == 0 && row == 0) record_status(P.status, VEDA_ERR_BAD_INDEX);
-                float mx = -INFINITY;
+                if (r.valid < TT) {                      // uniform: a short or out-of-range tile
+                    if (r.valid == 0 && row == 0) record_status(P.status, VEDA_ERR_BAD_INDEX);
 #pragma unroll
-                for (int c = 0; c < 128; ++c) {
-                    if (c >= r.valid) s[c] = __float_as_uint(-INFINITY);
-                    mx = fmaxf(mx, __uint_as_float(s[c]));
+                    for (int c = 0; c < 128; ++c)
+                        if (c >= r.valid) s[c] = __float_as_uint(-INFINITY);
                 }
+                // row max: eight independent 3-input chains, then a short tree
+                float a8[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) a8[k] = fmaxf(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1]));
+#pragma unroll
+                for (int base = 16; base < 128; base += 16)
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        a8[k] = max3f(a8[k], __uint_as_float(s[base + 2 * k]), __uint_as_float(s[base + 2 * k + 1]));
+                const float mx = fmaxf(max3f(a8[0], a8[1], a8[2]), max3f(max3f(a8[3], a8[4], a8[5]), a8[6], a8[7]));
                 const float mxs = mx * sl2;
                 bool rescale = false;
                 float alpha = 1.f;
@@ -449,26 +492,35 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                     }
                     m_run = mxs;
                 }
-                l *= alpha;
+                // a fully masked prefix leaves m_run = -inf; then every logit is -inf and p = 0
                 const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
+                const uint64_t scale2 = pk2(__float_as_uint(sl2), __float_as_uint(sl2));
+                const uint64_t negm2 = pk2(__float_as_uint(neg_m), __float_as_uint(neg_m));
 
                 const uint32_t pb = t & 1;
                 if (t >= 2 && !(ok = warp_wait(sm, &sm.p_free[pb], ((t >> 1) - 1) & 1, P.status))) break;
                 const uint32_t pa = tmem + lane_off + (pb ? kColP1 : kColP0);
+                uint64_t lsum[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     uint32_t packed[16];
 #pragma unroll
                     for (int c = 0; c < 16; ++c) {
-                        const float x0 = __uint_as_float(s[32 * q + 2 * c]);
-                        const float x1 = __uint_as_float(s[32 * q + 2 * c + 1]);
-                        const float p0 = (m_run == -INFINITY) ? 0.f : fast_exp2(fmaf(x0, sl2, neg_m));
-                        const float p1 = (m_run == -INFINITY) ? 0.f : fast_exp2(fmaf(x1, sl2, neg_m));
-                        l += p0 + p1;
+                        const uint64_t y = ffma2(pk2(s[32 * q + 2 * c], s[32 * q + 2 * c + 1]), scale2, negm2);
+                        float y0, y1;
+                        upk2(y, y0, y1);
+                        const float p0 = fast_exp2(y0), p1 = fast_exp2(y1);
+                        lsum[c & 3] = fadd2(lsum[c & 3], pk2(__float_as_uint(p0), __float_as_uint(p1)));
                         __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
                         packed[c] = *reinterpret_cast<uint32_t*>(&pr);
                     }
                     TMEM_ST16(pa + 16 * q, packed);
+                }
+                {
+                    const uint64_t t2 = fadd2(fadd2(lsum[0], lsum[1]), fadd2(lsum[2], lsum[3]));
+                    float s0, s1;
+                    upk2(t2, s0, s1);
+                    l = fmaf(l, alpha, s0 + s1);
                 }
                 tmem_wait_st();
                 // O holds the sum up to tile t-1 at the old max.  tcgen05.ld/st
