@@ -12,22 +12,25 @@
 //
 // Design (one CTA per SM, persistent, units in head-major order so the CTAs
 // in flight share one head's K/V in L2):
-//   warp 0      TMA producer: Q tile (double-buffered) and a 4-stage ring of
+//   warp 8      TMA producer: Q tile (double-buffered) and a 4-stage ring of
 //               32 KB K/V tiles, loaded in exactly the order the MMA warp
 //               consumes them: K0, K1, V0, K2, V1, ..., V(n-1).  Each tile is
 //               two 128-row x 128-byte boxes with the 128-byte swizzle.
-//   warp 1      MMA issuer (one thread): S(t+1) = Q K(t+1)^T is issued before
-//               O += P(t) V(t), so the tensor core works on the next score
-//               tile while the softmax warps exponentiate the current one.
-//   warp 2      TMEM allocator (all 512 columns).
-//   warps 4-7   softmax: thread = query row = TMEM lane.  Loads S from TMEM,
-//               masks keys past a segment's end, keeps a running max in
-//               base-2 units (rescaling O in TMEM only when the max grows by
-//               more than 2^8, otherwise the stale max is kept: the final
-//               division by the row sum makes the result exact either way),
-//               writes P as packed bf16 into TMEM (the A operand of P V), and
-//               finally normalises O and stores the row.
-// TMEM columns: S0 [0,128) S1 [128,256) P0 [256,320) P1 [320,384) O [384,512).
+//   warp 9      allocates TMEM; one thread issues the MMAs.  Kept tile j goes
+//               to softmax group g = j & 1: S(j) = Q K(j)^T into S buffer g,
+//               then O(g) += P(j) V(j) with P read from TMEM, and S(j+2) is
+//               issued right behind P(j) V(j) into the same buffer (the
+//               tensor pipe runs one thread's MMAs in issue order).
+//   warps 0-7   two softmax groups of four warps; warp % 4 is the TMEM lane
+//               quarter (thread = query row).  Each group takes every other
+//               kept tile, so the two groups run half a tile apart and one
+//               group's TMEM traffic overlaps the other's exponentials.  Per
+//               tile: load S, mask keys past a segment's end, running max in
+//               base-2 units with a lazy rescale of the group's O (only when
+//               the max grows by more than 2^8; the final division makes the
+//               stale max exact), P as packed bf16 over the S buffer.  The
+//               epilogue merges the two groups' (max, sum, O) and stores the
+//               rows (group g writes channels [64g, 64g + 64)).
 // Every mbarrier wait is bounded: on expiry the waiting thread records
 // VEDA_ERR_TIMEOUT in the status word and raises a CTA-wide abort flag; all
 // roles then leave their loops, outstanding TMA loads and MMAs are drained
@@ -46,8 +49,11 @@ constexpr int TT = 128;                   // tile rows (queries / keys)
 constexpr int NS = 4;                     // K/V ring stages
 constexpr int kTileBytes = TT * D * 2;    // 32 KB
 constexpr int kBoxBytes = kTileBytes / 2; // 128 rows x 128 bytes
-constexpr int kThreads = 256;
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColP0 = 256, kColP1 = 320, kColO = 384;
+constexpr int kThreads = 320;             // 10 warps: 8 softmax (two groups of 4), producer, MMA
+// TMEM columns: S of group g at 128*g (its P, packed bf16, aliases the first
+// 64 columns), O accumulator of group g at 256 + 128*g.
+__host__ __device__ constexpr uint32_t col_s(uint32_t g) { return 128u * g; }
+__host__ __device__ constexpr uint32_t col_o(uint32_t g) { return 256u + 128u * g; }
 constexpr long long kWaitLimit = 1ll << 31;   // clock cycles (~1 s)
 constexpr float kRescaleThreshold = 8.0f;     // log2 units: rescale O when the max grows > 2^8
 
@@ -71,7 +77,14 @@ struct __align__(1024) Smem {
     uint8_t q[2][kTileBytes];
     uint8_t kv[NS][kTileBytes];
     uint64_t q_full[2], q_empty[2], kv_full[NS], kv_empty[NS];
-    uint64_t s_full[2], s_free[2], p_full[2], p_free[2], drain;
+    uint64_t s_full[2];         // S of softmax group g ready in TMEM buffer g
+    uint64_t p_full[2];         // P of group g written (aliasing S buffer g)
+    uint64_t pv_done[2];        // P V of group g completed
+    uint64_t o_free;            // both O accumulators read by the epilogue
+    uint64_t xchg[4];           // per lane quarter: the two groups' (max, sum) exchanged
+    uint64_t drain;
+    float red_m[2][2][128];     // [unit parity][group][row] running max (base-2 units)
+    float red_l[2][2][128];     // [unit parity][group][row] running sum
     uint32_t tmem_base;
     volatile int abort_flag;
 };
@@ -318,26 +331,28 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int n_list = P.k_v + P.k_r + P.n_d;
+    constexpr int kProducerWarp = 8, kMmaWarp = 9;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sm.q_full[i], 1);
             mbar_init(&sm.q_empty[i], 1);
             mbar_init(&sm.s_full[i], 1);
-            mbar_init(&sm.s_free[i], 128);
             mbar_init(&sm.p_full[i], 128);
-            mbar_init(&sm.p_free[i], 1);
+            mbar_init(&sm.pv_done[i], 1);
         }
         for (int i = 0; i < NS; ++i) {
             mbar_init(&sm.kv_full[i], 1);
             mbar_init(&sm.kv_empty[i], 1);
         }
+        mbar_init(&sm.o_free, 256);
+        for (int q = 0; q < 4; ++q) mbar_init(&sm.xchg[q], 64);
         mbar_init(&sm.drain, 1);
         sm.abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
-    if (warp == 2) {
+    if (warp == kMmaWarp) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sm.tmem_base)),
                      "r"(512)
                      : "memory");
@@ -348,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
 
-    if (warp == 0 && lane == 0) {
+    if (warp == kProducerWarp && lane == 0) {
         // ------------------------------------------------ TMA producer ---
         uint32_t uq = 0, f = 0;
         bool ok = true;
@@ -371,6 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 ++f;
                 return true;
             };
+            // the MMA warp's consumption order: K0, K1, V0, K2, V1, ..., V(n-1)
             if (!(ok = load_kv(0, 0))) break;
             for (int j = 0; j < n_list && ok; ++j) {
                 if (j + 1 < n_list) ok = load_kv(j + 1, 0);
@@ -382,10 +398,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             if (!drain_phase(&sm.kv_full[k % NS], (k / NS) & 1, P.status)) break;
         for (uint32_t k = (uq > 2 ? uq - 2 : 0); k < uq; ++k)
             if (!drain_phase(&sm.q_full[k & 1], (k >> 1) & 1, P.status)) break;
-    } else if (warp == 1 && lane == 0) {
+    } else if (warp == kMmaWarp && lane == 0) {
         // ------------------------------------------------- MMA issuer ---
+        // Kept tile j goes to softmax group g = j & 1.  S(j+2) reuses group g's
+        // TMEM buffer, which holds P(j): it is issued right after P(j) V(j), and
+        // the tensor pipe runs one thread's MMAs in issue order.
         constexpr uint32_t idS = idesc_bf16(false), idPV = idesc_bf16(true);
-        uint32_t uq = 0, f = 0, ts = 0, tp = 0;
+        uint32_t uq = 0, f = 0, pc0 = 0, pc1 = 0, units_done = 0;
         bool ok = true;
         for (int64_t u = blockIdx.x; u < P.units && ok; u += gridDim.x) {
             const uint32_t qb = uq & 1;
@@ -393,78 +412,77 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             ++uq;
             tc_fence_after();
             const uint32_t qaddr = smem_u32(sm.q[qb]);
-            auto issue_s = [&]() -> bool {
-                const uint32_t st = f % NS, sb = ts & 1;
+            auto issue_s = [&](int j) -> bool {
+                const uint32_t st = f % NS, g = j & 1;
                 if (!wait_phase(sm, &sm.kv_full[st], (f / NS) & 1, P.status)) return false;
-                if (ts >= 2 && !wait_phase(sm, &sm.s_free[sb], ((ts >> 1) - 1) & 1, P.status)) return false;
                 tc_fence_after();
                 const uint32_t kaddr = smem_u32(sm.kv[st]);
-                const uint32_t d_tmem = tmem + (sb ? kColS1 : kColS0);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-                    umma_ss(d_tmem, smem_desc(qaddr + off, 16, 1024), smem_desc(kaddr + off, 16, 1024), idS,
+                    umma_ss(tmem + col_s(g), smem_desc(qaddr + off, 16, 1024), smem_desc(kaddr + off, 16, 1024), idS,
                             kk > 0);
                 }
-                umma_commit(&sm.s_full[sb]);
+                umma_commit(&sm.s_full[g]);
                 umma_commit(&sm.kv_empty[st]);
+                if (j == n_list - 1) umma_commit(&sm.q_empty[qb]);   // last read of this Q tile
                 ++f;
-                ++ts;
                 return true;
             };
-            if (!(ok = issue_s())) break;
+            if (!(ok = issue_s(0))) break;
+            if (n_list > 1 && !(ok = issue_s(1))) break;
             for (int j = 0; j < n_list && ok; ++j) {
-                if (j + 1 < n_list) {
-                    if (!(ok = issue_s())) break;
-                } else {
-                    umma_commit(&sm.q_empty[qb]);     // every S MMA of this unit has been issued
-                }
-                const uint32_t st = f % NS, pb = tp & 1;
+                const uint32_t g = j & 1, st = f % NS;
                 if (!(ok = wait_phase(sm, &sm.kv_full[st], (f / NS) & 1, P.status))) break;
-                if (!(ok = wait_phase(sm, &sm.p_full[pb], (tp >> 1) & 1, P.status))) break;
+                if (!(ok = wait_phase(sm, &sm.p_full[g], (g ? pc1 : pc0) & 1, P.status))) break;
+                if (j == 0 && units_done > 0 && !(ok = wait_phase(sm, &sm.o_free, (units_done - 1) & 1, P.status)))
+                    break;
                 tc_fence_after();
                 const uint32_t vaddr = smem_u32(sm.kv[st]);
-                const uint32_t p_tmem = tmem + (pb ? kColP1 : kColP0);
 #pragma unroll
                 for (int kk = 0; kk < TT / 16; ++kk)
-                    umma_ts(tmem + kColO, p_tmem + kk * 8, smem_desc(vaddr + kk * 2048, kBoxBytes, 1024), idPV,
-                            (j > 0 || kk > 0) ? 1u : 0u);
-                umma_commit(&sm.p_free[pb]);
+                    umma_ts(tmem + col_o(g), tmem + col_s(g) + kk * 8, smem_desc(vaddr + kk * 2048, kBoxBytes, 1024),
+                            idPV, (j >= 2 || kk > 0) ? 1u : 0u);
+                umma_commit(&sm.pv_done[g]);
                 umma_commit(&sm.kv_empty[st]);
                 ++f;
-                ++tp;
+                if (g) ++pc1; else ++pc0;
+                if (j + 2 < n_list && !(ok = issue_s(j + 2))) break;
             }
+            ++units_done;
         }
         // drain: all issued MMAs complete before TMEM is released
         umma_commit(&sm.drain);
         drain_phase(&sm.drain, 0, P.status);
-    } else if (warp >= 4) {
+    } else if (warp < 8) {
         // ---------------------------------------------------- softmax ---
-        const int wr = warp - 4;
-        const int row = wr * 32 + lane;
-        const uint32_t lane_off = (uint32_t)(wr * 32) << 16;
+        // Group g = warp / 4 takes kept tiles j = g, g+2, g+4, ...; warp % 4 is
+        // the TMEM lane quarter (thread = query row).  Each group keeps its own
+        // running max and sum and accumulates into its own O; the epilogue
+        // merges the two groups.
+        const int g = warp >> 2, wq = warp & 3;
+        const int row = wq * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
         const float sl2 = P.scale_log2;
-        uint32_t t = 0;
+        uint32_t sc = 0, uu = 0;          // S tiles consumed by this group; units done
         bool ok = true;
-        for (int64_t u = blockIdx.x; u < P.units && ok; u += gridDim.x) {
+        for (int64_t u = blockIdx.x; u < P.units && ok; u += gridDim.x, ++uu) {
             const int i = (int)(u % P.nq);
             const int64_t bh = u / P.nq;
             const int h = (int)(bh % P.H), b = (int)(bh / P.H);
             float m_run = -INFINITY, l = 0.f;
-            for (int j = 0; j < n_list; ++j, ++t) {
+            int cnt = 0;
+            for (int j = g; j < n_list; j += 2, ++sc, ++cnt) {
                 const TileRef r = resolve(P, u, j);      // index load overlaps the wait below
-                const uint32_t sb = t & 1;
-                if (!(ok = warp_wait(sm, &sm.s_full[sb], (t >> 1) & 1, P.status))) break;
+                if (!(ok = warp_wait(sm, &sm.s_full[g], sc & 1, P.status))) break;
                 tc_fence_after();
                 uint32_t s[128];
-                const uint32_t sa = tmem + lane_off + (sb ? kColS1 : kColS0);
+                const uint32_t sa = tmem + lane_off + col_s(g);
                 TMEM_LD32(sa + 0, (s + 0));
                 TMEM_LD32(sa + 32, (s + 32));
                 TMEM_LD32(sa + 64, (s + 64));
                 TMEM_LD32(sa + 96, (s + 96));
                 tmem_wait_ld();
-                tc_fence_before();
-                mbar_arrive(&sm.s_free[sb]);
 
                 if (r.valid < TT) {                      // uniform: a short or out-of-range tile
                     if (r.valid == 0 && row == 0) record_status(P.status, VEDA_ERR_BAD_INDEX);
@@ -488,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 if (mxs > m_run + kRescaleThreshold) {
                     if (m_run != -INFINITY) {
                         alpha = fast_exp2(m_run - mxs);
-                        rescale = (j > 0);
+                        rescale = (cnt > 0);
                     }
                     m_run = mxs;
                 }
@@ -497,9 +515,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 const uint64_t scale2 = pk2(__float_as_uint(sl2), __float_as_uint(sl2));
                 const uint64_t negm2 = pk2(__float_as_uint(neg_m), __float_as_uint(neg_m));
 
-                const uint32_t pb = t & 1;
-                if (t >= 2 && !(ok = warp_wait(sm, &sm.p_free[pb], ((t >> 1) - 1) & 1, P.status))) break;
-                const uint32_t pa = tmem + lane_off + (pb ? kColP1 : kColP0);
+                // P over the first 64 columns of the S buffer (S is in registers now;
+                // the previous P V of this group finished before this S was written)
                 uint64_t lsum[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
@@ -514,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                         __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
                         packed[c] = *reinterpret_cast<uint32_t*>(&pr);
                     }
-                    TMEM_ST16(pa + 16 * q, packed);
+                    TMEM_ST16(sa + 16 * q, packed);
                 }
                 {
                     const uint64_t t2 = fadd2(fadd2(lsum[0], lsum[1]), fadd2(lsum[2], lsum[3]));
@@ -523,16 +540,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                     l = fmaf(l, alpha, s0 + s1);
                 }
                 tmem_wait_st();
-                // O holds the sum up to tile t-1 at the old max.  tcgen05.ld/st
-                // are warp-collective, so when any row of this warp needs the
-                // rescale the whole warp waits for that product and rewrites its
-                // 32 rows of O (factor 1 for the rows that keep their max).
+                // This group's O holds its tiles before this one at the old max.
+                // tcgen05.ld/st are warp-collective: when any row of the warp needs
+                // the rescale, the whole warp waits for the group's previous P V and
+                // rewrites its 32 rows of O (factor 1 where the max is kept).
                 if (__any_sync(0xffffffffu, rescale)) {
-                    const uint32_t pp = (t - 1) & 1;
-                    if (!(ok = warp_wait(sm, &sm.p_free[pp], ((t - 1) >> 1) & 1, P.status))) break;
+                    if (!(ok = warp_wait(sm, &sm.pv_done[g], (sc - 1) & 1, P.status))) break;
                     tc_fence_after();
                     const float a = rescale ? alpha : 1.f;
-                    const uint32_t oa = tmem + lane_off + kColO;
+                    const uint32_t oa = tmem + lane_off + col_o(g);
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         uint32_t o[32];
@@ -545,31 +561,50 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                     tmem_wait_st();
                 }
                 tc_fence_before();
-                mbar_arrive(&sm.p_full[pb]);
+                mbar_arrive(&sm.p_full[g]);
             }
             if (!ok) break;
 
-            // ---- epilogue: O / l, bf16, one row per thread ----
-            const uint32_t tl = t - 1;
-            if (!(ok = warp_wait(sm, &sm.p_free[tl & 1], (tl >> 1) & 1, P.status))) break;
+            // ---- epilogue: merge the two groups; group g stores channels [64g, 64g+64) ----
+            if (cnt > 0 && !(ok = warp_wait(sm, &sm.pv_done[g], (sc - 1) & 1, P.status))) break;
+            const uint32_t up = uu & 1;
+            sm.red_m[up][g][row] = m_run;
+            sm.red_l[up][g][row] = l;
+            mbar_arrive(&sm.xchg[wq]);
+            if (!(ok = warp_wait(sm, &sm.xchg[wq], uu & 1, P.status))) break;
             tc_fence_after();
+            const float m0 = sm.red_m[up][0][row], m1 = sm.red_m[up][1][row];
+            const float l0 = sm.red_l[up][0][row], l1 = sm.red_l[up][1][row];
+            const float M = fmaxf(m0, m1);
+            const float f0 = (m0 == -INFINITY) ? 0.f : fast_exp2(m0 - M);
+            const float f1 = (m1 == -INFINITY) ? 0.f : fast_exp2(m1 - M);
+            const float L = l0 * f0 + l1 * f1;
+            const float inv = 1.f / L;
+            const float c0 = f0 * inv, c1 = f1 * inv;
             const int64_t tok = (int64_t)i * TT + row;
-            const float inv = 1.f / l;
-            const uint32_t oa = tmem + lane_off + kColO;
-            __nv_bfloat16* dst = P.out + (((int64_t)b * P.n_tok[0] + tok) * P.H + h) * D;
+            __nv_bfloat16* dst = P.out + (((int64_t)b * P.n_tok[0] + tok) * P.H + h) * D + 64 * g;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                uint32_t o[32];
-                TMEM_LD32(oa + 32 * q, o);
+            for (int q = 0; q < 2; ++q) {
+                uint32_t o0[32], o1[32];
+                TMEM_LD32(tmem + lane_off + col_o(0) + 64 * g + 32 * q, o0);
+                TMEM_LD32(tmem + lane_off + col_o(1) + 64 * g + 32 * q, o1);
                 tmem_wait_ld();
                 if (tok < P.n_tok[0]) {
 #pragma unroll
                     for (int c = 0; c < 32; c += 8) {
+                        float v[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            // a group with no tile in this unit contributes nothing
+                            // (its O holds stale values: never multiplied in)
+                            const float a0 = __uint_as_float(o0[c + e]) * c0;
+                            v[e] = (c1 != 0.f) ? fmaf(__uint_as_float(o1[c + e]), c1, a0) : a0;
+                        }
                         uint4 w;
-                        __nv_bfloat162 v0 = __floats2bfloat162_rn(__uint_as_float(o[c]) * inv, __uint_as_float(o[c + 1]) * inv);
-                        __nv_bfloat162 v1 = __floats2bfloat162_rn(__uint_as_float(o[c + 2]) * inv, __uint_as_float(o[c + 3]) * inv);
-                        __nv_bfloat162 v2 = __floats2bfloat162_rn(__uint_as_float(o[c + 4]) * inv, __uint_as_float(o[c + 5]) * inv);
-                        __nv_bfloat162 v3 = __floats2bfloat162_rn(__uint_as_float(o[c + 6]) * inv, __uint_as_float(o[c + 7]) * inv);
+                        __nv_bfloat162 v0 = __floats2bfloat162_rn(v[0], v[1]);
+                        __nv_bfloat162 v1 = __floats2bfloat162_rn(v[2], v[3]);
+                        __nv_bfloat162 v2 = __floats2bfloat162_rn(v[4], v[5]);
+                        __nv_bfloat162 v3 = __floats2bfloat162_rn(v[6], v[7]);
                         w.x = *reinterpret_cast<uint32_t*>(&v0);
                         w.y = *reinterpret_cast<uint32_t*>(&v1);
                         w.z = *reinterpret_cast<uint32_t*>(&v2);
@@ -578,9 +613,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                     }
                 }
             }
-            if (P.lse && tok < P.n_tok[0])
-                P.lse[((int64_t)b * P.H + h) * P.n_tok[0] + tok] = (m_run + __log2f(l)) * 0.69314718055994531f;
+            if (P.lse && g == 0 && tok < P.n_tok[0])
+                P.lse[((int64_t)b * P.H + h) * P.n_tok[0] + tok] = (M + __log2f(L)) * 0.69314718055994531f;
             tc_fence_before();
+            mbar_arrive(&sm.o_free);
         }
     }
 
@@ -588,7 +624,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 2) {
+    if (warp == kMmaWarp) {
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512) : "memory");
     }
 }

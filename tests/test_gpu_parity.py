@@ -142,6 +142,7 @@ REDUCED = {
                                     dense=(("text", 130), ("vlm", 70), ("audio", 64))),
     "portrait_boost": lambda: _reduced("portrait_10.13s", frames=5, Y=21, X=16, budget_video=4),
     "t2v_no_dense": lambda: _reduced("t2v_5.17s", dense=(), budget_video=2),
+    "t2v_single_tile": lambda: _reduced("t2v_5.17s", dense=(), budget_video=1),
     "fp32_d128": lambda: _reduced("t2v_5.17s", dtype="f32"),
     "bf16_d64_t64": lambda: _reduced("t2v_5.17s", d=64, T=64, r=32, budget_video=5),
 }
