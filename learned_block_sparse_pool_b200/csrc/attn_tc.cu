@@ -472,8 +472,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             const int h = (int)(bh % P.H), b = (int)(bh / P.H);
             float m_run = -INFINITY, l = 0.f;
             int cnt = 0;
+            TileRef r_next = resolve(P, u, g);
             for (int j = g; j < n_list; j += 2, ++sc, ++cnt) {
-                const TileRef r = resolve(P, u, j);      // index load overlaps the wait below
+                const TileRef r = r_next;
+                if (j + 2 < n_list) r_next = resolve(P, u, j + 2);   // one tile ahead
                 if (!(ok = warp_wait(sm, &sm.s_full[g], sc & 1, P.status))) break;
                 tc_fence_after();
                 uint32_t s[128];
