@@ -153,6 +153,16 @@ def oracle_sample(w, g, heads=2, units=16, seed=0):
 
 # ---------------------------------------------------------------------------
 
+def max_over_ranks(dist, values, device):
+    """Element-wise max of a list of floats over all ranks (no-op when not
+    distributed)."""
+    if dist is None:
+        return list(values)
+    t = torch.tensor(list(values), device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
 def make_problem(veda, w, g, simt=False):
     return veda.Problem(g["q"], g["k"], g["v"], tile=w.T, r=w.r, budget=w.budget_video,
                         k_ref=g.get("k_ref"), v_ref=g.get("v_ref"),
@@ -166,6 +176,15 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        # the CPU oracle: rank 0 alone runs and prints; other ranks do no work
+        if rank == 0:
+            w = workloads.get(args.workload)
+            if args.budget:
+                w = w.with_budget(args.budget)
+            dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
+            run_reference(args, w, dev, world)
+        return
     dist = None
     if world > 1:
         import torch.distributed as dist
@@ -180,13 +199,6 @@ def main():
     if args.heads:
         w = workloads.small(w.name, H=args.heads, budget_video=w.budget_video)
     n = world
-
-    if args.impl == "reference":
-        if rank == 0:
-            run_reference(args, w, dev, n)
-        if dist is not None:
-            dist.destroy_process_group()
-        return
 
     import learned_block_sparse_pool_b200 as veda
     g = workloads.make_inputs(w, device=dev)
@@ -240,10 +252,7 @@ def main():
     total_ms = t_start.elapsed_time(t_end)
     stage = [[evs[k][s].elapsed_time(evs[k][s + 1]) for k in range(args.steps)] for s in range(4)]
     stage_avg = [sum(x) / len(x) for x in stage]
-    if dist is not None:
-        t = torch.tensor([total_ms] + stage_avg, device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, *stage_avg = t.tolist()
+    total_ms, *stage_avg = max_over_ranks(dist, [total_ms] + stage_avg, dev)
 
     pk, pk_src = peaks()
     attn_s = stage_avg[3] / 1e3
@@ -345,11 +354,7 @@ def e2e_run(veda, w, g, p, dev, stream, steps, n, dist, simt):
         one()
     t1.record(stream)
     torch.cuda.synchronize(dev)
-    ms = t0.elapsed_time(t1)
-    if dist is not None:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = t.item()
+    ms = max_over_ranks(dist, [t0.elapsed_time(t1)], dev)[0]
     st = veda.check_status(ws, stream)
     if st != 0:
         raise RuntimeError(f"device status after e2e: {veda.status_string(st)}")
@@ -360,7 +365,7 @@ def e2e_run(veda, w, g, p, dev, stream, steps, n, dist, simt):
 def run_reference(args, w, dev, n):
     """--impl reference: the CPU oracle on the host cores, each step a bounded
     sample of the same workload, extrapolated to ms per call."""
-    g = workloads.make_inputs(w, device=dev if torch.cuda.is_available() else "cpu")
+    g = workloads.make_inputs(w, device=dev)
     for _ in range(args.warmup):
         oracle_sample(w, g, heads=2, units=8)
     vals = []

@@ -79,6 +79,13 @@ typedef enum { VEDA_F32 = 0, VEDA_BF16 = 1 } veda_dtype;
 #define VEDA_FLAG_SIMT_ATTENTION 1u /* run attention on the fp32 SIMT kernel even
                                        where the tensor-core kernel applies (bf16,
                                        d = 128, tile = 128): a cross-check path  */
+#define VEDA_FLAG_TEST_SHORT_WAITS 2u /* test hook for the failure path: the
+                                       tensor-core attention kernel's pipeline
+                                       waits give up after ~64 clocks, so the
+                                       call stops early, frees its resources and
+                                       reports VEDA_ERR_TIMEOUT through
+                                       veda_check_status(); its output is then
+                                       undefined.  No effect on other kernels. */
 
 /* One key/value segment, [B, n_tokens, H, d] (d contiguous). */
 typedef struct {

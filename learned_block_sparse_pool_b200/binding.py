@@ -25,6 +25,7 @@ VEDA_ERR_TIMEOUT = -5
 VEDA_ERR_BAD_INDEX = -6
 VEDA_F32, VEDA_BF16 = 0, 1
 VEDA_FLAG_SIMT_ATTENTION = 1
+VEDA_FLAG_TEST_SHORT_WAITS = 2
 
 EXPORTS = ("veda_workspace_size", "veda_workspace_init", "veda_select_tiles", "veda_block_sparse_attn",
            "veda_attn", "veda_pool_project", "veda_score_tiles", "veda_topk_tiles", "veda_workspace_view",

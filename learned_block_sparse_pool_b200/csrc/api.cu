@@ -73,7 +73,7 @@ veda_status validate(const veda_problem* pp)
     if (p.tile != 64 && p.tile != 128) return VEDA_ERR_UNSUPPORTED;
     if (p.r > 128 || p.r % 4 != 0) return VEDA_ERR_UNSUPPORTED;
     if (!(p.softmax_scale >= 0.f) || !isfinite(p.softmax_scale)) return VEDA_ERR_INVALID_ARG;
-    if (p.flags & ~VEDA_FLAG_SIMT_ATTENTION) return VEDA_ERR_INVALID_ARG;
+    if (p.flags & ~(VEDA_FLAG_SIMT_ATTENTION | VEDA_FLAG_TEST_SHORT_WAITS)) return VEDA_ERR_INVALID_ARG;
     if (!p.q || !aligned16(p.q)) return VEDA_ERR_INVALID_ARG;
     const size_t es = esize(p.dtype);
     if (!stride_ok(p.q_stride_b, es) || !stride_ok(p.q_stride_tok, es) || !stride_ok(p.q_stride_h, es))
@@ -223,6 +223,7 @@ veda_status do_attn(const veda_problem& p, const Layout& L, const int32_t* idx_v
     A.dtype = p.dtype;
     A.scale = p.softmax_scale > 0.f ? p.softmax_scale : 1.0f / sqrtf((float)p.d);
     A.status = at<uint32_t>(ws, 0);
+    A.short_waits = (p.flags & VEDA_FLAG_TEST_SHORT_WAITS) ? 1 : 0;
     if (!(p.flags & VEDA_FLAG_SIMT_ATTENTION) && attn_tc_supported(A)) return from_cuda(launch_attn_tc(A, s));
     return from_cuda(launch_attn_simt(A, s));
 }

@@ -71,6 +71,7 @@ struct TcParams {
     float* lse;
     float scale_log2;
     uint32_t* status;
+    long long wait_limit;       // clocks a pipeline wait may take before the CTA aborts
 };
 
 struct __align__(1024) Smem {
@@ -125,14 +126,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* b, uint32_t parity)
 }
 
 // Bounded wait: true when the phase completed, false on timeout or abort.
-__device__ __forceinline__ bool wait_phase(Smem& sm, uint64_t* b, uint32_t parity, uint32_t* status)
+__device__ __forceinline__ bool wait_phase(Smem& sm, uint64_t* b, uint32_t parity, uint32_t* status,
+                                           long long limit)
 {
     if (mbar_try_wait(b, parity)) return true;
     const long long t0 = clock64();
     for (;;) {
         if (mbar_try_wait(b, parity)) return true;
         if (sm.abort_flag) return false;
-        if (clock64() - t0 > kWaitLimit) {
+        if (clock64() - t0 > limit) {
             record_status(status, VEDA_ERR_TIMEOUT);
             sm.abort_flag = 1;
             return false;
@@ -142,9 +144,10 @@ __device__ __forceinline__ bool wait_phase(Smem& sm, uint64_t* b, uint32_t parit
 
 // Wait by every lane of a warp that next issues warp-collective tcgen05.ld /
 // tcgen05.st: reconverges the warp and makes the outcome warp-uniform.
-__device__ __forceinline__ bool warp_wait(Smem& sm, uint64_t* b, uint32_t parity, uint32_t* status)
+__device__ __forceinline__ bool warp_wait(Smem& sm, uint64_t* b, uint32_t parity, uint32_t* status,
+                                          long long limit)
 {
-    const bool ok = wait_phase(sm, b, parity, status);
+    const bool ok = wait_phase(sm, b, parity, status, limit);
     return __all_sync(0xffffffffu, ok);
 }
 
@@ -372,14 +375,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             const int64_t bh = u / P.nq;
             const int h = (int)(bh % P.H), b = (int)(bh / P.H);
             const uint32_t qb = uq & 1;
-            if (uq >= 2 && !(ok = wait_phase(sm, &sm.q_empty[qb], ((uq >> 1) - 1) & 1, P.status))) break;
+            if (uq >= 2 && !(ok = wait_phase(sm, &sm.q_empty[qb], ((uq >> 1) - 1) & 1, P.status, P.wait_limit))) break;
             mbar_expect_tx(&sm.q_full[qb], kTileBytes);
             load_box_pair(P, 0, sm.q[qb], &sm.q_full[qb], h, i * TT, b);
             ++uq;
             auto load_kv = [&](int j, int which) -> bool {
                 const TileRef r = resolve(P, u, j);
                 const uint32_t st = f % NS;
-                if (f >= NS && !wait_phase(sm, &sm.kv_empty[st], ((f / NS) - 1) & 1, P.status)) return false;
+                if (f >= NS && !wait_phase(sm, &sm.kv_empty[st], ((f / NS) - 1) & 1, P.status, P.wait_limit)) return false;
                 mbar_expect_tx(&sm.kv_full[st], kTileBytes);
                 const int tok = r.valid > 0 ? r.tile * TT : (int)P.n_tok[r.seg];
                 load_box_pair(P, 1 + 2 * r.seg + which, sm.kv[st], &sm.kv_full[st], h, tok, b);
@@ -408,13 +411,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         bool ok = true;
         for (int64_t u = blockIdx.x; u < P.units && ok; u += gridDim.x) {
             const uint32_t qb = uq & 1;
-            if (!(ok = wait_phase(sm, &sm.q_full[qb], (uq >> 1) & 1, P.status))) break;
+            if (!(ok = wait_phase(sm, &sm.q_full[qb], (uq >> 1) & 1, P.status, P.wait_limit))) break;
             ++uq;
             tc_fence_after();
             const uint32_t qaddr = smem_u32(sm.q[qb]);
             auto issue_s = [&](int j) -> bool {
                 const uint32_t st = f % NS, g = j & 1;
-                if (!wait_phase(sm, &sm.kv_full[st], (f / NS) & 1, P.status)) return false;
+                if (!wait_phase(sm, &sm.kv_full[st], (f / NS) & 1, P.status, P.wait_limit)) return false;
                 tc_fence_after();
                 const uint32_t kaddr = smem_u32(sm.kv[st]);
 #pragma unroll
@@ -433,9 +436,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             if (n_list > 1 && !(ok = issue_s(1))) break;
             for (int j = 0; j < n_list && ok; ++j) {
                 const uint32_t g = j & 1, st = f % NS;
-                if (!(ok = wait_phase(sm, &sm.kv_full[st], (f / NS) & 1, P.status))) break;
-                if (!(ok = wait_phase(sm, &sm.p_full[g], (g ? pc1 : pc0) & 1, P.status))) break;
-                if (j == 0 && units_done > 0 && !(ok = wait_phase(sm, &sm.o_free, (units_done - 1) & 1, P.status)))
+                if (!(ok = wait_phase(sm, &sm.kv_full[st], (f / NS) & 1, P.status, P.wait_limit))) break;
+                if (!(ok = wait_phase(sm, &sm.p_full[g], (g ? pc1 : pc0) & 1, P.status, P.wait_limit))) break;
+                if (j == 0 && units_done > 0 && !(ok = wait_phase(sm, &sm.o_free, (units_done - 1) & 1, P.status, P.wait_limit)))
                     break;
                 tc_fence_after();
                 const uint32_t vaddr = smem_u32(sm.kv[st]);
@@ -476,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             for (int j = g; j < n_list; j += 2, ++sc, ++cnt) {
                 const TileRef r = r_next;
                 if (j + 2 < n_list) r_next = resolve(P, u, j + 2);   // one tile ahead
-                if (!(ok = warp_wait(sm, &sm.s_full[g], sc & 1, P.status))) break;
+                if (!(ok = warp_wait(sm, &sm.s_full[g], sc & 1, P.status, P.wait_limit))) break;
                 tc_fence_after();
                 uint32_t s[128];
                 const uint32_t sa = tmem + lane_off + col_s(g);
@@ -547,7 +550,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 // the rescale, the whole warp waits for the group's previous P V and
                 // rewrites its 32 rows of O (factor 1 where the max is kept).
                 if (__any_sync(0xffffffffu, rescale)) {
-                    if (!(ok = warp_wait(sm, &sm.pv_done[g], (sc - 1) & 1, P.status))) break;
+                    if (!(ok = warp_wait(sm, &sm.pv_done[g], (sc - 1) & 1, P.status, P.wait_limit))) break;
                     tc_fence_after();
                     const float a = rescale ? alpha : 1.f;
                     const uint32_t oa = tmem + lane_off + col_o(g);
@@ -568,12 +571,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             if (!ok) break;
 
             // ---- epilogue: merge the two groups; group g stores channels [64g, 64g+64) ----
-            if (cnt > 0 && !(ok = warp_wait(sm, &sm.pv_done[g], (sc - 1) & 1, P.status))) break;
+            if (cnt > 0 && !(ok = warp_wait(sm, &sm.pv_done[g], (sc - 1) & 1, P.status, P.wait_limit))) break;
             const uint32_t up = uu & 1;
             sm.red_m[up][g][row] = m_run;
             sm.red_l[up][g][row] = l;
             mbar_arrive(&sm.xchg[wq]);
-            if (!(ok = warp_wait(sm, &sm.xchg[wq], uu & 1, P.status))) break;
+            if (!(ok = warp_wait(sm, &sm.xchg[wq], uu & 1, P.status, P.wait_limit))) break;
             tc_fence_after();
             const float m0 = sm.red_m[up][0][row], m1 = sm.red_m[up][1][row];
             const float l0 = sm.red_l[up][0][row], l1 = sm.red_l[up][1][row];
@@ -732,6 +735,7 @@ cudaError_t launch_attn_tc(const AttnParams& a, cudaStream_t s)
     P.lse = a.lse;
     P.scale_log2 = a.scale * 1.4426950408889634f;
     P.status = a.status;
+    P.wait_limit = a.short_waits ? 64 : kWaitLimit;
 
     const size_t smem = sizeof(Smem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -14,8 +14,9 @@
 // the (job, b, h, tile) items in order; each CTA owns one contiguous run of
 // items, so it loads W[h] into shared memory once per head it meets.  Within
 // a tile, each thread owns one 16-byte column chunk of the row and a set of
-// tokens: every warp load is a 128-bit, fully coalesced access, and all of a
-// thread's loads for the tile are issued before any is consumed.
+// tokens: every warp load is a 128-bit, fully coalesced access; all of a
+// thread's loads for the next tile are issued before this tile is reduced and
+// projected, so HBM traffic overlaps the arithmetic.
 #include <cuda_bf16.h>
 
 #include "veda_internal.cuh"
@@ -78,18 +79,39 @@ __global__ void __launch_bounds__(kThreads) pool_project_kernel(const PoolParams
 
     const int64_t it0 = (int64_t)blockIdx.x * P.total_items / gridDim.x;
     const int64_t it1 = (int64_t)(blockIdx.x + 1) * P.total_items / gridDim.x;
+    if (it0 >= it1) return;
+    // decode the first item of this CTA's run once; later items are stepped to
+    int j = 0;
+    while (j + 1 < P.n_jobs && it0 >= P.job[j + 1].first_item) ++j;
+    int i, h, b;
+    {
+        const int64_t local = it0 - P.job[j].first_item;
+        i = (int)(local % P.job[j].n_tiles);
+        const int64_t bh = local / P.job[j].n_tiles;
+        h = (int)(bh % P.H);
+        b = (int)(bh / P.H);
+    }
     int cur_job = -1, cur_h = -1;
 
-    for (int64_t it = it0; it < it1; ++it) {
-        int j = 0;
-        while (j + 1 < P.n_jobs && it >= P.job[j + 1].first_item) ++j;
-        const PoolJob& J = P.job[j];
-        const int64_t local = it - J.first_item;
-        const int i = (int)(local % J.n_tiles);
-        const int64_t bh = local / J.n_tiles;
-        const int h = (int)(bh % P.H);
-        const int b = (int)(bh / P.H);
+    // one thread's 16-byte loads of its column chunk for a tile; issued one
+    // item ahead so the next tile streams in while this one is reduced
+    uint4 raw[LOADS];
+    auto issue = [&](int jj, int bb, int hh, int ii) {
+        const PoolJob& J = P.job[jj];
+        const int64_t t0 = (int64_t)ii * P.T;
+        const int64_t t1 = min(J.n_tokens, t0 + P.T);
+        const Tin* base = static_cast<const Tin*>(J.x) + (int64_t)bb * J.sb + (int64_t)hh * J.sh +
+                          (int64_t)chunk * EPC;
+#pragma unroll
+        for (int u = 0; u < LOADS; ++u) {
+            const int64_t t = t0 + row0 + (int64_t)u * RP;
+            raw[u] = (t < t1) ? load_stream(base + t * J.st) : make_uint4(0u, 0u, 0u, 0u);
+        }
+    };
+    issue(j, b, h, i);
 
+    for (int64_t it = it0; it < it1; ++it) {
+        const PoolJob& J = P.job[j];
         if (j != cur_job || h != cur_h) {
             __syncthreads();   // the previous item's projection no longer reads w_s
             const Tin* W = static_cast<const Tin*>(J.w) + (int64_t)h * D * r;
@@ -97,18 +119,10 @@ __global__ void __launch_bounds__(kThreads) pool_project_kernel(const PoolParams
             cur_job = j;
             cur_h = h;
         }
+        const int64_t t0 = (int64_t)i * P.T;
+        const int cnt = (int)(min(J.n_tokens, t0 + P.T) - t0);
 
         // ---- pool: sum this thread's tokens of its 16-byte column chunk ----
-        const int64_t t0 = (int64_t)i * P.T;
-        const int64_t t1 = min(J.n_tokens, t0 + P.T);
-        const Tin* base = static_cast<const Tin*>(J.x) + (int64_t)b * J.sb + (int64_t)h * J.sh +
-                          (int64_t)chunk * EPC;
-        uint4 raw[LOADS];
-#pragma unroll
-        for (int u = 0; u < LOADS; ++u) {
-            const int64_t t = t0 + row0 + (int64_t)u * RP;
-            raw[u] = (t < t1) ? load_stream(base + t * J.st) : make_uint4(0u, 0u, 0u, 0u);
-        }
         float acc[EPC];
 #pragma unroll
         for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
@@ -119,6 +133,20 @@ __global__ void __launch_bounds__(kThreads) pool_project_kernel(const PoolParams
 #pragma unroll
             for (int e = 0; e < EPC; ++e) acc[e] += f[e];
         }
+        // this item's coordinates, then the next item's loads
+        const int ci = i, ch = h, cb = b;
+        if (++i == J.n_tiles) {
+            i = 0;
+            if (++h == P.H) {
+                h = 0;
+                if (++b == P.B) {
+                    b = 0;
+                    ++j;
+                }
+            }
+        }
+        if (it + 1 < it1) issue(j, b, h, i);
+
 #pragma unroll
         for (int e = 0; e < EPC; ++e) part[row0 * D + chunk * EPC + e] = acc[e];
         __syncthreads();
@@ -126,7 +154,7 @@ __global__ void __launch_bounds__(kThreads) pool_project_kernel(const PoolParams
             float s = 0.f;
 #pragma unroll 8
             for (int q = 0; q < RP; ++q) s += part[q * D + tid];
-            pooled[tid] = s / (float)(t1 - t0);
+            pooled[tid] = s / (float)cnt;
         }
         __syncthreads();
 
@@ -142,7 +170,7 @@ __global__ void __launch_bounds__(kThreads) pool_project_kernel(const PoolParams
         if (tid < r) {
             float s = 0.f;
             for (int q = 0; q < groups; ++q) s += proj[q * r + tid];
-            J.out[((int64_t)(b * P.H + h) * J.n_tiles + i) * r + tid] = s;
+            J.out[((int64_t)(cb * P.H + ch) * J.n_tiles + ci) * r + tid] = s;
         }
     }
 }

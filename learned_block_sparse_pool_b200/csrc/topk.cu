@@ -9,22 +9,19 @@
 //
 // Algorithm (exact; no sorting):
 //   1. The warp loads its row once (coalesced 4-byte lanes, all loads in
-//      flight) into registers, with the row's min and max.
-//   2. A 256-bucket histogram over a monotone linear map of [min, max]
-//      locates the bucket b* holding the k-th largest score.  Buckets are
-//      monotone in the value, so every element of a higher bucket is
-//      strictly larger than every element of b*, and equal values share a
-//      bucket.
-//   3. The few elements of b* are compacted to shared memory and an 8-bit
-//      radix select over their order-preserving 32-bit keys finds the exact
-//      k-th largest key tau and how many elements equal to tau are still
-//      needed.  (If b* holds too many elements -- near-constant rows -- the
-//      radix select runs over the whole row instead.)
-//   4. One pass in index order emits key > tau, plus the first `need` keys
+//      flight) into registers as order-preserving 32-bit keys, and reduces
+//      the row's smallest and largest key.
+//   2. Radix select on the key bits below the row's common prefix (the bits
+//      where the smallest and largest key agree are shared by every key), 8
+//      bits at a time, most significant first: a 256-bin shared-memory
+//      histogram locates the digit holding the k-th largest key.  After the
+//      first digit the (few) keys still matching the prefix are compacted to
+//      shared memory and the remaining digits are resolved over them only.
+//      The result is the exact k-th largest key tau and how many keys equal
+//      to tau are still needed.
+//   3. One pass in index order emits key > tau, plus the first `need` keys
 //      equal to tau: warp ballots give each lane its output slot, so the
 //      list is written ascending and coalesced.
-// -0.0 and +0.0 are one key (a tie); NaN ranks below every number.
-#include <float.h>
 
 #include "veda_internal.cuh"
 
@@ -90,118 +87,105 @@ __device__ __forceinline__ void clear_hist(uint32_t* hist, int lane)
     __syncwarp();
 }
 
-template <int PL>   // elements per lane held in registers (n <= 32 * PL)
+// One warp per row; the row's keys live in this warp's slice of dynamic
+// shared memory (lane-strided: key e at keys[e]).
 __global__ void __launch_bounds__(32 * kWarps) topk_kernel(const TopkParams P)
 {
-    __shared__ uint32_t hist_s[kWarps][NB];
-    __shared__ uint32_t cand_s[kWarps][kCandMax];
+    extern __shared__ uint32_t smem[];
     const int lane = threadIdx.x & 31;
     const int w = threadIdx.x >> 5;
-    uint32_t* hist = hist_s[w];
-    uint32_t* cand = cand_s[w];
-    const uint32_t lt_mask = (1u << lane) - 1u;
     const int n = P.n;
+    const int nkeys = (n + 31) & ~31;
+    uint32_t* hist = smem + (size_t)w * (NB + kCandMax + nkeys);
+    uint32_t* cand = hist + NB;
+    uint32_t* keys = cand + kCandMax;
+    const uint32_t lt_mask = (1u << lane) - 1u;
 
     for (int64_t row = (int64_t)blockIdx.x * kWarps + w; row < P.rows;
          row += (int64_t)gridDim.x * kWarps) {
         const float* src = P.scores + row * P.ld;
-        float v[PL];
-#pragma unroll
-        for (int m = 0; m < PL; ++m) {
-            const int e = lane + 32 * m;
-            v[m] = (e < n) ? __ldcs(src + e) : 0.f;
+        // ---- load: keys to shared memory, smallest and largest key ----
+        uint32_t kmin = 0xffffffffu, kmax = 0u;
+#pragma unroll 8
+        for (int e = lane; e < n; e += 32) {
+            const uint32_t kk = order_key(__ldcs(src + e));
+            keys[e] = kk;
+            kmin = min(kmin, kk);
+            kmax = max(kmax, kk);
         }
-        float lo = FLT_MAX, hi = -FLT_MAX;
-#pragma unroll
-        for (int m = 0; m < PL; ++m) {
-            const int e = lane + 32 * m;
-            if (e < n && v[m] == v[m]) {
-                lo = fminf(lo, v[m]);
-                hi = fmaxf(hi, v[m]);
-            }
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
-            hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
-        }
-        float sc = 0.f;
-        if (hi > lo) {
-            const float range = hi - lo;
-            if (range < FLT_MAX) sc = ((float)NB * 0.999999f) / range;
-        }
-
-        // ---- 2. bucket histogram ----
-        clear_hist(hist, lane);
-#pragma unroll
-        for (int m = 0; m < PL; ++m) {
-            const int e = lane + 32 * m;
-            if (e < n) {
-                const float f = (v[m] == v[m]) ? v[m] : lo;
-                const int bk = min(NB - 1, max(0, (int)((f - lo) * sc)));
-                atomicAdd(&hist[bk], 1u);
-            }
-        }
+        kmin = __reduce_min_sync(0xffffffffu, kmin);
+        kmax = __reduce_max_sync(0xffffffffu, kmax);
         __syncwarp();
-        int above = 0;
-        const int bstar = find_digit_from_top(hist, P.k, lane, &above);
-        int rem = P.k - above;          // kept elements still to take from bucket b*
 
-        // ---- 3. candidates of b*, exact k-th key by radix select ----
-        int nc = 0;
-#pragma unroll
-        for (int m = 0; m < PL; ++m) {
-            const int e = lane + 32 * m;
-            bool in = false;
-            if (e < n) {
-                const float f = (v[m] == v[m]) ? v[m] : lo;
-                in = min(NB - 1, max(0, (int)((f - lo) * sc))) == bstar;
-            }
-            const uint32_t bal = __ballot_sync(0xffffffffu, in);
-            const int pos = nc + __popc(bal & lt_mask);
-            if (in && pos < kCandMax) cand[pos] = order_key(v[m]);
-            nc += __popc(bal);
-        }
-        __syncwarp();
-        const bool small = nc <= kCandMax;
-        uint32_t prefix = 0u, pmask = 0u;
-        if (!small) rem = P.k;          // fall back: radix select over the whole row
-#pragma unroll 1
-        for (int shift = 24; shift >= 0; shift -= 8) {
+        uint32_t tau;
+        int need;
+        if (kmin == kmax) {            // every key equal: the first k indices
+            tau = kmin;
+            need = P.k;
+        } else {
+            const int top = 31 - __clz(kmin ^ kmax);             // highest bit where keys differ
+            uint32_t pmask = top == 31 ? 0u : ~((1u << (top + 1)) - 1u);
+            uint32_t prefix = kmin & pmask;                       // shared by every key
+            int rem = P.k;
+            int shift = top >= 7 ? top - 7 : 0;
+            // ---- first digit over the whole row ----
             clear_hist(hist, lane);
-            if (small) {
-                for (int c = lane; c < nc; c += 32) {
-                    const uint32_t key = cand[c];
-                    if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
-                }
-            } else {
-#pragma unroll
-                for (int m = 0; m < PL; ++m) {
-                    const int e = lane + 32 * m;
-                    const uint32_t key = order_key(v[m]);
-                    if (e < n && (key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
-                }
+#pragma unroll 4
+            for (int e = lane; e < n; e += 32) atomicAdd(&hist[(keys[e] >> shift) & 255u], 1u);
+            __syncwarp();
+            {
+                int ab = 0;
+                const int dg = find_digit_from_top(hist, rem, lane, &ab);
+                rem -= ab;
+                pmask |= 255u << shift;
+                prefix = (prefix & ~(255u << shift)) | ((uint32_t)dg << shift);
+            }
+            // ---- compact the keys that still match ----
+            int nc = 0;
+            for (int base = 0; base < n; base += 32) {
+                const int e = base + lane;
+                const uint32_t kk = e < n ? keys[e] : 0u;
+                const bool in = (e < n) && (kk & pmask) == prefix;
+                const uint32_t bal = __ballot_sync(0xffffffffu, in);
+                const int pos = nc + __popc(bal & lt_mask);
+                if (in && pos < kCandMax) cand[pos] = kk;
+                nc += __popc(bal);
             }
             __syncwarp();
-            int ab = 0;
-            const int dgt = find_digit_from_top(hist, rem, lane, &ab);
-            rem -= ab;
-            prefix |= (uint32_t)dgt << shift;
-            pmask |= 255u << shift;
+            const bool small = nc <= kCandMax;
+            const uint32_t* pool = small ? cand : keys;
+            const int npool = small ? nc : n;
+            // ---- remaining digits, over the candidates (or the row) ----
+#pragma unroll 1
+            while (shift > 0) {
+                const int nshift = shift >= 8 ? shift - 8 : 0;
+                const uint32_t dmask = (1u << (shift - nshift)) - 1u;
+                clear_hist(hist, lane);
+                for (int c = lane; c < npool; c += 32) {
+                    const uint32_t kk = pool[c];
+                    if ((kk & pmask) == prefix) atomicAdd(&hist[(kk >> nshift) & dmask], 1u);
+                }
+                __syncwarp();
+                int ab = 0;
+                const int dg = find_digit_from_top(hist, rem, lane, &ab);
+                rem -= ab;
+                pmask |= dmask << nshift;
+                prefix |= (uint32_t)dg << nshift;
+                shift = nshift;
+            }
+            tau = prefix;
+            need = rem;
         }
-        const uint32_t tau = prefix;
-        const int need = rem;           // keys equal to tau to keep, lowest index first
 
-        // ---- 4. emit in index order ----
+        // ---- emit in index order: key > tau, then the first `need` keys == tau ----
         int32_t* dst = P.idx + row * (int64_t)P.k;
         int out = 0, eq_seen = 0;
-#pragma unroll
-        for (int m = 0; m < PL; ++m) {
-            const int e = lane + 32 * m;
-            const uint32_t key = order_key(v[m]);
+        for (int base = 0; base < n && out < P.k; base += 32) {
+            const int e = base + lane;
+            const uint32_t kk = e < n ? keys[e] : 0u;
             const bool valid = e < n;
-            const bool gt = valid && key > tau;
-            const bool eq = valid && key == tau;
+            const bool gt = valid && kk > tau;
+            const bool eq = valid && kk == tau;
             const uint32_t eqb = __ballot_sync(0xffffffffu, eq);
             const bool sel = gt || (eq && eq_seen + __popc(eqb & lt_mask) < need);
             const uint32_t selb = __ballot_sync(0xffffffffu, sel);
@@ -214,19 +198,7 @@ __global__ void __launch_bounds__(32 * kWarps) topk_kernel(const TopkParams P)
     }
 }
 
-template <int PL>
-cudaError_t launch_pl(const TopkParams& p, cudaStream_t s)
-{
-    int per_sm = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, topk_kernel<PL>, 32 * kWarps, 0);
-    if (e != cudaSuccess) return e;
-    if (per_sm < 1) per_sm = 1;
-    int64_t grid = (int64_t)num_sms() * per_sm;
-    const int64_t need = (p.rows + kWarps - 1) / kWarps;
-    if (grid > need) grid = need;
-    topk_kernel<PL><<<(unsigned)grid, 32 * kWarps, 0, s>>>(p);
-    return cudaGetLastError();
-}
+size_t topk_smem_bytes(int n) { return sizeof(uint32_t) * (size_t)kWarps * (NB + kCandMax + ((n + 31) & ~31)); }
 
 }  // namespace
 
@@ -235,13 +207,19 @@ int topk_max_tiles() { return 32 * 128; }
 cudaError_t launch_topk(const TopkParams& p, cudaStream_t s)
 {
     if (p.rows == 0) return cudaSuccess;
-    if (p.n <= 32 * 4) return launch_pl<4>(p, s);
-    if (p.n <= 32 * 16) return launch_pl<16>(p, s);
-    if (p.n <= 32 * 32) return launch_pl<32>(p, s);
-    if (p.n <= 32 * 64) return launch_pl<64>(p, s);
-    if (p.n <= 32 * 96) return launch_pl<96>(p, s);
-    if (p.n <= 32 * 128) return launch_pl<128>(p, s);
-    return cudaErrorInvalidValue;
+    if (p.n > topk_max_tiles()) return cudaErrorInvalidValue;
+    const size_t smem = topk_smem_bytes(p.n);
+    cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, topk_kernel, 32 * kWarps, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) per_sm = 1;
+    int64_t grid = (int64_t)num_sms() * per_sm;
+    const int64_t need = (p.rows + kWarps - 1) / kWarps;
+    if (grid > need) grid = need;
+    topk_kernel<<<(unsigned)grid, 32 * kWarps, smem, s>>>(p);
+    return cudaGetLastError();
 }
 
 }  // namespace veda

@@ -84,6 +84,7 @@ struct AttnParams {
     int32_t dtype;
     float scale;            // softmax scale (natural-log units)
     uint32_t* status;
+    int32_t short_waits;    // test hook: bounded waits give up after ~64 clocks
 };
 
 cudaError_t launch_attn_simt(const AttnParams& p, cudaStream_t s);

@@ -110,7 +110,7 @@ def test_valid_problem_workspace_size(L):
     ({"r": 132}, B.VEDA_ERR_UNSUPPORTED),
     ({"B": 0}, B.VEDA_ERR_INVALID_ARG),
     ({"dtype": 7}, B.VEDA_ERR_INVALID_ARG),
-    ({"flags": 2}, B.VEDA_ERR_INVALID_ARG),
+    ({"flags": 4}, B.VEDA_ERR_INVALID_ARG),
     ({"softmax_scale": -1.0}, B.VEDA_ERR_INVALID_ARG),
     ({"softmax_scale": float("nan")}, B.VEDA_ERR_INVALID_ARG),
     ({"q": 0}, B.VEDA_ERR_INVALID_ARG),
@@ -131,6 +131,12 @@ def test_valid_problem_workspace_size(L):
 def test_invalid_arguments_rejected_on_host(L, over, code):
     st, _ = _ws_size(L, _problem(**over))
     assert st == code, (over, B.status_string(st))
+
+
+def test_test_hook_flags_are_accepted(L):
+    for flags in (B.VEDA_FLAG_SIMT_ATTENTION, B.VEDA_FLAG_TEST_SHORT_WAITS, 3):
+        st, _ = _ws_size(L, _problem(flags=flags))
+        assert st == B.VEDA_OK
 
 
 def test_optional_segments_absent_is_valid(L):

@@ -218,6 +218,28 @@ def test_out_of_range_index_is_flagged(dev, simt):
     assert veda.check_status(ws) == 0            # reading re-arms the status word
 
 
+def test_wait_timeout_is_reported_and_the_context_recovers(dev, oracle_mod):
+    """Failure path of the tensor-core kernel: with the short-wait test hook
+    every pipeline wait gives up almost at once; the kernel must drain what it
+    started, free TMEM, return, and report VEDA_ERR_TIMEOUT.  A normal call on
+    the same context afterwards must still be correct."""
+    w = _reduced("t2v_5.17s")
+    inp = workloads.make_inputs(w)
+    g = to_dev(inp, dev)
+    p = make_problem(w, g)
+    ws = veda.workspace(p)
+    iv, ir = gpu_select(p, g, ws)
+    assert veda.check_status(ws) == 0
+    bad = make_problem(w, g, flags=veda.binding.VEDA_FLAG_TEST_SHORT_WAITS)
+    out, _ = veda.alloc_output(bad)
+    for _ in range(2):
+        veda.block_sparse_attn(bad, iv, ir, out, None, ws)
+        assert veda.check_status(ws) == veda.binding.VEDA_ERR_TIMEOUT
+    sel = oracle_mod.select_tiles(inp, w.T, w.budget_video)
+    units = [(0, h, i) for h in range(w.H) for i in range(w.n_q_tiles)]
+    check_attention(oracle_mod, w, inp, p, ws, sel, units, "after timeouts")
+
+
 def test_simt_and_default_paths_agree(dev):
     w = _reduced("r2va_5.17s", ref_frames=1, budget_ref=2)
     g = to_dev(workloads.make_inputs(w), dev)
