@@ -14,9 +14,10 @@
 // the (job, b, h, tile) items in order; each CTA owns one contiguous run of
 // items, so it loads W[h] into shared memory once per head it meets.  Within
 // a tile, each thread owns one 16-byte column chunk of the row and a set of
-// tokens: every warp load is a 128-bit, fully coalesced access; all of a
-// thread's loads for the next tile are issued before this tile is reduced and
-// projected, so HBM traffic overlaps the arithmetic.
+// tokens: every warp load is a 128-bit, fully coalesced access, and a tile's
+// loads are issued before the previous tile is summed.  Up to four
+// consecutive tiles of a head are pooled per round and reduced and projected
+// together, so the per-tile barrier and projection overhead stays small.
 #include <cuda_bf16.h>
 
 #include "veda_internal.cuh"
@@ -57,6 +58,8 @@ __device__ __forceinline__ uint4 load_stream(const void* p)
     return v;
 }
 
+constexpr int kGroup = 4;   // tiles of one head pooled per round
+
 template <typename Tin, int D>
 __global__ void __launch_bounds__(kThreads) pool_project_kernel(const PoolParams P)
 {
@@ -68,14 +71,12 @@ __global__ void __launch_bounds__(kThreads) pool_project_kernel(const PoolParams
     extern __shared__ float smem[];
     const int r = P.r;
     float* w_s = smem;                         // [D][r]
-    float* part = w_s + D * r;                 // [RP][D]
-    float* pooled = part + RP * D;             // [D]
-    float* proj = pooled + D;                  // [groups][r]
+    float* part = w_s + D * r;                 // [kGroup][RP][D]
+    float* pooled = part + kGroup * RP * D;    // [kGroup][D]
 
     const int tid = threadIdx.x;
     const int chunk = tid % CPR;
     const int row0 = tid / CPR;
-    const int groups = kThreads / r;
 
     const int64_t it0 = (int64_t)blockIdx.x * P.total_items / gridDim.x;
     const int64_t it1 = (int64_t)(blockIdx.x + 1) * P.total_items / gridDim.x;
@@ -93,84 +94,86 @@ __global__ void __launch_bounds__(kThreads) pool_project_kernel(const PoolParams
     }
     int cur_job = -1, cur_h = -1;
 
-    // one thread's 16-byte loads of its column chunk for a tile; issued one
-    // item ahead so the next tile streams in while this one is reduced
+    // one thread's 16-byte loads of its column chunk for one tile
     uint4 raw[LOADS];
-    auto issue = [&](int jj, int bb, int hh, int ii) {
-        const PoolJob& J = P.job[jj];
-        const int64_t t0 = (int64_t)ii * P.T;
-        const int64_t t1 = min(J.n_tokens, t0 + P.T);
-        const Tin* base = static_cast<const Tin*>(J.x) + (int64_t)bb * J.sb + (int64_t)hh * J.sh +
-                          (int64_t)chunk * EPC;
+    auto issue = [&](const PoolJob& J, int bb, int hh, int ii) {
+        const int t0 = ii * P.T;
+        const int cnt = (int)min((int64_t)P.T, J.n_tokens - (int64_t)t0);
+        const char* base = reinterpret_cast<const char*>(J.x) +
+                           ((int64_t)bb * J.sb + (int64_t)hh * J.sh + (int64_t)(t0 + row0) * J.st + chunk * EPC) *
+                               (int64_t)sizeof(Tin);
+        const int64_t step = (int64_t)RP * J.st * (int64_t)sizeof(Tin);
 #pragma unroll
-        for (int u = 0; u < LOADS; ++u) {
-            const int64_t t = t0 + row0 + (int64_t)u * RP;
-            raw[u] = (t < t1) ? load_stream(base + t * J.st) : make_uint4(0u, 0u, 0u, 0u);
-        }
+        for (int u = 0; u < LOADS; ++u)
+            raw[u] = (row0 + u * RP < cnt) ? load_stream(base + u * step) : make_uint4(0u, 0u, 0u, 0u);
     };
-    issue(j, b, h, i);
 
-    for (int64_t it = it0; it < it1; ++it) {
+    int64_t it = it0;
+    issue(P.job[j], b, h, i);
+    while (it < it1) {
         const PoolJob& J = P.job[j];
         if (j != cur_job || h != cur_h) {
-            __syncthreads();   // the previous item's projection no longer reads w_s
+            __syncthreads();   // the previous round's projection no longer reads w_s
             const Tin* W = static_cast<const Tin*>(J.w) + (int64_t)h * D * r;
             for (int e = tid; e < D * r; e += kThreads) w_s[e] = to_f32(W[e]);
             cur_job = j;
             cur_h = h;
         }
-        const int64_t t0 = (int64_t)i * P.T;
-        const int cnt = (int)(min(J.n_tokens, t0 + P.T) - t0);
-
-        // ---- pool: sum this thread's tokens of its 16-byte column chunk ----
-        float acc[EPC];
+        // a round: up to kGroup consecutive tiles of this (job, b, h)
+        const int i0 = i;
+        const int ng = (int)min((int64_t)kGroup, min((int64_t)(J.n_tiles - i0), it1 - it));
+        for (int g = 0; g < ng; ++g) {
+            float acc[EPC];
 #pragma unroll
-        for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
+            for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
 #pragma unroll
-        for (int u = 0; u < LOADS; ++u) {
-            float f[EPC];
-            unpack(raw[u], f, (const Tin*)nullptr);
+            for (int u = 0; u < LOADS; ++u) {
+                float f[EPC];
+                unpack(raw[u], f, (const Tin*)nullptr);
 #pragma unroll
-            for (int e = 0; e < EPC; ++e) acc[e] += f[e];
-        }
-        // this item's coordinates, then the next item's loads
-        const int ci = i, ch = h, cb = b;
-        if (++i == J.n_tiles) {
-            i = 0;
-            if (++h == P.H) {
-                h = 0;
-                if (++b == P.B) {
-                    b = 0;
-                    ++j;
+                for (int e = 0; e < EPC; ++e) acc[e] += f[e];
+            }
+            // next tile's loads go out before this one's partial sums are stored
+            int ni = i + 1, nh = h, nb = b, nj = j;
+            if (ni == J.n_tiles) {
+                ni = 0;
+                if (++nh == P.H) {
+                    nh = 0;
+                    if (++nb == P.B) {
+                        nb = 0;
+                        ++nj;
+                    }
                 }
             }
-        }
-        if (it + 1 < it1) issue(j, b, h, i);
-
+            if (it + 1 < it1) issue(P.job[nj], nb, nh, ni);
+            float* dst = part + (g * RP + row0) * D + chunk * EPC;
 #pragma unroll
-        for (int e = 0; e < EPC; ++e) part[row0 * D + chunk * EPC + e] = acc[e];
+            for (int e = 0; e < EPC; ++e) dst[e] = acc[e];
+            i = ni; h = nh; b = nb; j = nj;
+            ++it;
+        }
         __syncthreads();
-        if (tid < D) {
+        // pooled means of the round's tiles
+        for (int x = tid; x < ng * D; x += kThreads) {
+            const int g = x / D, e = x % D;
+            const int t0 = (i0 + g) * P.T;
+            const int cnt = (int)min((int64_t)P.T, J.n_tokens - (int64_t)t0);
             float s = 0.f;
 #pragma unroll 8
-            for (int q = 0; q < RP; ++q) s += part[q * D + tid];
-            pooled[tid] = s / (float)cnt;
+            for (int q = 0; q < RP; ++q) s += part[(g * RP + q) * D + e];
+            pooled[g * D + e] = s / (float)cnt;
         }
         __syncthreads();
-
-        // ---- project: xhat[c] = sum_e pooled[e] * W[h][e][c] ----
-        const int c = tid % r;
-        const int g = tid / r;
-        if (g < groups) {
+        // projection of the round's pooled vectors: one output (g, c) per thread
+        const int hh = cur_h;
+        const int bb = (int)(((it - ng - J.first_item) / J.n_tiles) / P.H);
+        for (int x = tid; x < ng * r; x += kThreads) {
+            const int g = x / r, c = x % r;
+            const float* pv = pooled + g * D;
             float s = 0.f;
-            for (int e = g; e < D; e += groups) s += pooled[e] * w_s[e * r + c];
-            proj[g * r + c] = s;
-        }
-        __syncthreads();
-        if (tid < r) {
-            float s = 0.f;
-            for (int q = 0; q < groups; ++q) s += proj[q * r + tid];
-            J.out[((int64_t)(cb * P.H + ch) * J.n_tiles + ci) * r + tid] = s;
+#pragma unroll 8
+            for (int e = 0; e < D; ++e) s = fmaf(pv[e], w_s[e * r + c], s);
+            J.out[((int64_t)(bb * P.H + hh) * J.n_tiles + i0 + g) * r + c] = s;
         }
     }
 }
@@ -180,8 +183,7 @@ cudaError_t launch_typed(const PoolParams& p, cudaStream_t s)
 {
     constexpr int EPC = 16 / sizeof(Tin);
     constexpr int RP = kThreads / (D / EPC);
-    const int groups = kThreads / p.r;
-    const size_t smem = sizeof(float) * ((size_t)D * p.r + RP * D + D + (size_t)groups * p.r);
+    const size_t smem = sizeof(float) * ((size_t)D * p.r + (size_t)kGroup * RP * D + (size_t)kGroup * D);
     auto kern = pool_project_kernel<Tin, D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

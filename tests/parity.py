@@ -5,6 +5,13 @@ Tolerances (stated once, used by every parity test):
     score within TIE_REL (relative, in the oracle's fp64) of the row's k-th
     score -- a near-tie the fp32 kernels may legitimately order either way;
     every such row is reported.
+  * selector projections q̂, k̂ (fp32 on the device): each element within
+    the forward error bound of fp32 summation (Higham, "Accuracy and
+    Stability of Numerical Algorithms", section 3.1: a sum of n terms in any
+    order is off by at most gamma_(n-1) times the sum of the terms' magnitudes,
+    gamma_n = n u / (1 - n u), u = 2^-24).  The tile mean (T terms, one
+    division) and the projection (d multiply-adds) together give
+    |err_c| <= (gamma_(T+1) + gamma_(d+1)) * sum_e |W[e, c]| * mean_t |x[t, e]|.
   * attention, fp32 problems: max-abs <= 1e-4 and relative L2 <= 1e-4.
   * attention, bf16 problems: max-abs <= 2e-2 and relative L2 <= 5e-3
     (the output itself is rounded to bf16, 2^-9 relative).
@@ -19,6 +26,25 @@ import torch
 
 TIE_REL = 1e-4
 TOL = {torch.float32: (1e-4, 1e-4), torch.bfloat16: (2e-2, 5e-3)}
+
+
+U32 = 2.0 ** -24
+
+
+def gamma(n: int) -> float:
+    return n * U32 / (1.0 - n * U32)
+
+
+def assert_projection_within_bound(oracle_mod, got: np.ndarray, want: np.ndarray, x: torch.Tensor,
+                                   w: torch.Tensor, T: int, what: str = ""):
+    """got: the device's fp32 projection [B,H,n,r]; want: the oracle's fp64;
+    x: the pooled input [B,N,H,d]; w: the weights [H,d,r]."""
+    d = x.shape[-1]
+    mag = oracle_mod.project(oracle_mod.pool(x.abs(), T), w.abs())
+    bound = (gamma(T + 1) + gamma(d + 1)) * mag
+    err = np.abs(got - want)
+    worst = float(np.max(err / np.maximum(bound, 1e-300)))
+    assert worst <= 1.0, f"{what}: projection error {worst:.3g} x the fp32 summation bound"
 
 
 @dataclass

@@ -21,7 +21,8 @@ import torch
 
 import learned_block_sparse_pool_b200 as veda
 import workloads
-from parity import assert_close, assert_selection, compare_selection, gather_lse, gather_units
+from parity import (assert_close, assert_projection_within_bound, assert_selection, compare_selection,
+                    gather_lse, gather_units)
 
 pytestmark = pytest.mark.gpu
 
@@ -53,12 +54,13 @@ def gpu_select(p, g, ws):
     return iv, ir
 
 
-def check_selection(oracle_mod, p, ws, iv, ir, sel, what):
-    r = p.c.r
-    qh = veda.workspace_view(p, ws, 0)[..., :r].double().cpu().numpy()
-    kh = veda.workspace_view(p, ws, 1)[..., :r].double().cpu().numpy()
-    np.testing.assert_allclose(qh, sel["qhat"], rtol=2e-5, atol=2e-6)
-    np.testing.assert_allclose(kh, sel["khat"], rtol=2e-5, atol=2e-6)
+def check_selection(oracle_mod, p, ws, iv, ir, sel, what, inp):
+    r, T = p.c.r, p.c.tile
+    for which, name, x, w in ((0, "qhat", "q", "w_q"), (1, "khat", "k", "w_k"), (2, "khat_r", "k_ref", "w_k")):
+        if name not in sel:
+            continue
+        got = veda.workspace_view(p, ws, which)[..., :r].double().cpu().numpy()
+        assert_projection_within_bound(oracle_mod, got, sel[name], inp[x], inp[w], T, f"{what} {name}")
     rep = compare_selection(oracle_mod, iv.cpu().numpy(), sel["idx_v"], sel["kth_v"], sel["qhat"], sel["khat"])
     assert_selection(rep, what + " video")
     if ir is not None:
@@ -97,7 +99,7 @@ def test_tiny_workload(dev, oracle_mod):
     ws = veda.workspace(p)
     iv, ir = gpu_select(p, g, ws)
     sel = oracle_mod.select_tiles(inp, w.T, w.budget_video)
-    check_selection(oracle_mod, p, ws, iv, ir, sel, "tiny")
+    check_selection(oracle_mod, p, ws, iv, ir, sel, "tiny", inp)
     units = [(0, h, i) for h in range(w.H) for i in range(w.n_q_tiles)]
     out, err = check_attention(oracle_mod, w, inp, p, ws, sel, units, "tiny attention")
     print(f"tiny: max-abs {err[0]:.3g} rel-L2 {err[1]:.3g}")
@@ -158,7 +160,7 @@ def test_reduced_workloads(dev, oracle_mod, name, simt):
     ws = veda.workspace(p)
     iv, ir = gpu_select(p, g, ws)
     sel = oracle_mod.select_tiles(inp, w.T, w.budget_video, w.budget_ref if w.ref_frames else 0)
-    check_selection(oracle_mod, p, ws, iv, ir, sel, name)
+    check_selection(oracle_mod, p, ws, iv, ir, sel, name, inp)
     units = [(0, h, i) for h in range(w.H) for i in range(w.n_q_tiles)]
     check_attention(oracle_mod, w, inp, p, ws, sel, units, name)
 
@@ -179,7 +181,7 @@ def test_budget_every_tile_and_budget_one(dev, oracle_mod, dtype):
         ws = veda.workspace(p)
         iv, ir = gpu_select(p, g, ws)
         sel = oracle_mod.select_tiles(inp, w.T, k)
-        check_selection(oracle_mod, p, ws, iv, ir, sel, f"budget {k}")
+        check_selection(oracle_mod, p, ws, iv, ir, sel, f"budget {k}", inp)
         units = [(0, h, i) for h in range(w.H) for i in range(n)]
         check_attention(oracle_mod, wk, inp, p, ws, sel, units, f"budget {k}")
 
@@ -197,7 +199,7 @@ def test_batch_two_non_packed_strides(dev, oracle_mod):
     ws = veda.workspace(p)
     iv, ir = gpu_select(p, g, ws)
     sel = oracle_mod.select_tiles(inp, w.T, w.budget_video, w.budget_ref)
-    check_selection(oracle_mod, p, ws, iv, ir, sel, "batch2")
+    check_selection(oracle_mod, p, ws, iv, ir, sel, "batch2", inp)
     units = [(b, h, i) for b in range(2) for h in range(w.H) for i in range(w.n_q_tiles)]
     check_attention(oracle_mod, w, inp, p, ws, sel, units, "batch2")
 
@@ -281,7 +283,7 @@ def test_full_size_workload(dev, oracle_mod, name):
     torch.cuda.synchronize()
     host = {k: v.cpu() for k, v in g.items()}
     sel = oracle_mod.select_tiles(host, w.T, w.budget_video, w.budget_ref if w.ref_frames else 0)
-    rep = check_selection(oracle_mod, p, ws, iv, ir, sel, name)
+    rep = check_selection(oracle_mod, p, ws, iv, ir, sel, name, host)
     print(f"{name}: {rep.rows} selection rows, {len(rep.tie_band)} inside the tie band")
     units = sample_units(w)
     _, err = check_attention(oracle_mod, w, host, p, ws, sel, units, name)
