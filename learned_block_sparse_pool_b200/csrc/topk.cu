@@ -7,20 +7,27 @@
 // "How the SN120 Competition Works"; veyrul.com, "Veda R2VA for MiniMax-H3",
 // second paragraph: 32 reference + 32 video tiles chosen independently).
 //
-// Algorithm (exact; no sorting), one warp per row:
-//   1. Bracket: 256 keys sampled at a fixed stride give a lower bound `lo`
-//      that, with a 3-sigma margin, at least k keys of the row reach.
-//   2. One streaming pass over the row (coalesced loads, many in flight)
-//      keeps every key >= lo, with its index, in a small candidate list in
-//      shared memory, in index order.
+// Algorithm (exact; no sorting), one warp per row, on order-preserving
+// 32-bit keys of the scores:
+//   1. Bracket: 256 keys sampled at a fixed stride are binned linearly in key
+//      space (one shared-memory histogram); the lower edge `lo` of the bin
+//      holding the sample rank of the k-th largest key plus a 3-sigma margin
+//      is a bound that, with high probability, at least k keys reach.
+//   2. One streaming pass over the row (float4 loads, issued together with
+//      the sample's) keeps every key >= lo, with its index, in a candidate
+//      list in shared memory, in index order.
 //   3. If at least k keys were kept (and the list did not overflow), the
-//      top-k set and every key tied with its smallest member are among them:
-//      an 8-bit radix select over the candidates' order-preserving keys finds
-//      the k-th largest key tau and how many keys equal to tau are still
-//      needed, and one ballot pass over the candidates emits the kept indices
-//      in ascending order (ties to the lowest index).  Otherwise (a skewed or
-//      tied row) the same radix select runs over the whole row, re-read from
-//      global memory, followed by an emit pass over the row.
+//      top-k set and every key tied with its smallest member are among them.
+//      The candidates are binned linearly between their smallest and largest
+//      key; the bin b holding the k-th largest key is found from the
+//      histogram, and the (at most 32) keys of bin b are ranked exactly
+//      against each other, which gives the k-th largest key tau and how
+//      many keys equal to tau are taken.  (A bin of more than 32 keys --
+//      heavy ties -- falls back to an 8-bit radix select over the
+//      candidates.)  One ballot pass over the candidates then emits the kept
+//      indices in ascending order, ties to the lowest index.  If the bracket
+//      missed, a radix select runs over the whole row, re-read from global
+//      memory, followed by an emit pass over the row.
 // The sample only decides how much work is done, never which tiles are kept.
 // -0.0 and +0.0 are one key (a tie); NaN ranks below every number.
 #include <algorithm>
@@ -90,7 +97,8 @@ __device__ __forceinline__ void clear_hist(uint32_t* hist, int lane)
 }
 
 constexpr int kSample = 256;
-constexpr int kCapMax = 2048;   // candidate-list capacity bound (shared memory)
+constexpr int kCapMax = 2048;
+constexpr int kChunk = 512;     // keys per streaming step of a warp (float4 per lane x 128)   // candidate-list capacity bound (shared memory)
 
 // Radix select over `cnt` keys provided by get(c) (c in [0, cnt)), all in
 // [kmin, kmax]: returns the key tau of rank `rank` (0 = largest) and, through
@@ -131,6 +139,79 @@ __device__ __forceinline__ uint32_t radix_rank(Get get, int cnt, int rank, uint3
 __device__ __forceinline__ uint32_t warp_min(uint32_t x) { return __reduce_min_sync(0xffffffffu, x); }
 __device__ __forceinline__ uint32_t warp_max(uint32_t x) { return __reduce_max_sync(0xffffffffu, x); }
 
+// Inverse of order_key for keys of numbers.
+__device__ __forceinline__ float key_value(uint32_t k)
+{
+    return __uint_as_float((k & 0x80000000u) ? (k ^ 0x80000000u) : ~k);
+}
+
+// Linear bins in value between two finite values lo < hi: bin(v) =
+// min(255, floor((v - lo) * 256 / (hi - lo))), non-decreasing in v (each step
+// rounds monotonically).  `ok` is false when the range is not finite.
+struct Bins {
+    float lo, scale;
+    bool ok;
+    __device__ __forceinline__ Bins(uint32_t kmin, uint32_t kmax)
+    {
+        lo = key_value(kmin);
+        const float hi = key_value(kmax);
+        scale = 256.f / (hi - lo);
+        ok = kmin != 0u && isfinite(lo) && isfinite(hi) && isfinite(scale) && scale > 0.f;
+    }
+    __device__ __forceinline__ uint32_t operator()(uint32_t k) const
+    {
+        return min(255u, (uint32_t)((key_value(k) - lo) * scale));
+    }
+};
+
+// The k-th largest of `cnt` candidate keys (cnt >= k), all in [kmin, kmax],
+// kmin < kmax: one histogram over linear value bins locates the bin holding
+// it, and the bin's keys are ranked exactly against each other.  Returns
+// false when the range is not finite or that bin holds more than 32 keys.  On success *tau is
+// the k-th largest key and *need the number of keys equal to tau among the
+// k largest (taking every key > tau and the first *need keys == tau in
+// candidate order gives exactly k keys).
+__device__ __forceinline__ bool bin_select(const uint32_t* ckey, int cnt, int k, uint32_t kmin, uint32_t kmax,
+                                           uint32_t* hist, int lane, uint32_t* tau, int* need)
+{
+    const Bins bin(kmin, kmax);
+    if (!bin.ok) return false;
+    clear_hist(hist, lane);
+    for (int c = lane; c < cnt; c += 32) atomicAdd(&hist[bin(ckey[c])], 1u);
+    __syncwarp();
+    int above = 0;
+    const uint32_t b = (uint32_t)find_digit_from_top(hist, k, lane, &above);
+    const int nb = (int)hist[b];
+    __syncwarp();                                   // every lane has read the histogram
+    if (nb > 32) return false;
+    // gather bin b's keys (candidate order) into hist[0 .. nb)
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    int pos = 0;
+    for (int cb = 0; cb < cnt && pos < nb; cb += 32) {
+        const int c = cb + lane;
+        const uint32_t kk = c < cnt ? ckey[c] : 0u;
+        const bool in = c < cnt && bin(kk) == b;
+        const uint32_t bal = __ballot_sync(0xffffffffu, in);
+        if (in) hist[pos + __popc(bal & lt_mask)] = kk;
+        pos += __popc(bal);
+    }
+    __syncwarp();
+    const int nb_need = k - above;                  // keys still to take from bin b (>= 1)
+    const uint32_t mine = lane < nb ? hist[lane] : 0u;
+    int gt = 0, ge = 0;
+    for (int t = 0; t < nb; ++t) {
+        const uint32_t x = hist[t];
+        gt += x > mine;
+        ge += x >= mine;
+    }
+    const uint32_t hit = __ballot_sync(0xffffffffu, lane < nb && gt < nb_need && nb_need <= ge);
+    const int src = __ffs(hit) - 1;                 // some key of the bin has this rank
+    *tau = __shfl_sync(0xffffffffu, mine, src);
+    *need = nb_need - __shfl_sync(0xffffffffu, gt, src);
+    __syncwarp();
+    return true;
+}
+
 // Lower bracket rank in a sample of kSample keys for budget k of n: the
 // expected sample rank of the k-th largest key plus three standard deviations
 // (binomial) and a small constant.
@@ -144,18 +225,15 @@ __host__ __device__ __forceinline__ int bracket_rank(int n, int k)
 }
 
 // One warp per row.  Per-warp shared memory: histogram | candidate keys
-// (cap) | candidate indices (cap); the sample (kSample keys) is held in the
-// candidate region before the candidates are written.
-__global__ void __launch_bounds__(32 * kWarps) topk_kernel(const TopkParams P, int cap, int r_lo)
+// (cap) | candidate indices (cap).
+__global__ void __launch_bounds__(32 * kWarps, 4) topk_kernel(const TopkParams P, int cap, int r_lo)
 {
     extern __shared__ uint32_t smem[];
     const int lane = threadIdx.x & 31;
     const int w = threadIdx.x >> 5;
     const int n = P.n, k = P.k;
-    const int region = cap * 2 > kSample ? cap * 2 : kSample;
-    uint32_t* hist = smem + (size_t)w * (NB + region);
+    uint32_t* hist = smem + (size_t)w * (NB + 2 * cap);
     uint32_t* ckey = hist + NB;
-    uint32_t* samp = ckey;
     int32_t* cidx = reinterpret_cast<int32_t*>(ckey + cap);
     const uint32_t lt_mask = (1u << lane) - 1u;
     const bool sampled = n > kSample && r_lo < kSample - 1;
@@ -170,48 +248,70 @@ __global__ void __launch_bounds__(32 * kWarps) topk_kernel(const TopkParams P, i
             continue;
         }
 
-        // ---- 1. bracket from a strided sample ----
-        uint32_t lo = 0u;                   // 0: keep everything
-        if (sampled) {
-            uint32_t smin = 0xffffffffu, smax = 0u;
+        // ---- 1. loads of the first kChunk keys and of the strided sample ----
+        // lane L holds keys 128u + 4L .. 128u + 4L + 3 of each kChunk-key chunk
+        float4 v[kChunk / 128];
+        auto load_chunk = [&](int base) {
 #pragma unroll
-            for (int m = 0; m < kSample / 32; ++m) {
-                const int sidx = (int)(((int64_t)(lane + 32 * m) * n) / kSample);
-                const uint32_t kk = order_key(__ldg(src + sidx));
-                samp[lane + 32 * m] = kk;
-                smin = min(smin, kk);
-                smax = max(smax, kk);
-            }
-            smin = warp_min(smin);
-            smax = warp_max(smax);
-            __syncwarp();
-            int dummy = 0;
-            lo = radix_rank([&](int c) { return samp[c]; }, kSample, r_lo, smin, smax, hist, lane, &dummy);
-        }
-
-        // ---- 2. streaming pass: keys >= lo, with indices, in index order ----
-        // chunks of 1024 keys: lane L holds keys 128u + 4L .. 128u + 4L + 3
-        int nc = 0;
-        uint32_t cmax = 0u, cmin = 0xffffffffu;
-        for (int base = 0; base < n; base += 1024) {
-            float4 v[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
+            for (int u = 0; u < kChunk / 128; ++u) {
                 const int e = base + 128 * u + 4 * lane;
                 v[u] = e < n ? __ldcs(reinterpret_cast<const float4*>(src + e))
                              : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
             }
+        };
+        load_chunk(0);
+        uint32_t lo = 0u;                   // 0: keep everything
+        if (sampled) {
+            uint32_t sk[kSample / 32];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
+            for (int m = 0; m < kSample / 32; ++m) sk[m] = order_key(__ldg(src + ((lane + 32 * m) * n) / kSample));
+            uint32_t smin = sk[0], smax = sk[0];
+#pragma unroll
+            for (int m = 1; m < kSample / 32; ++m) {
+                smin = min(smin, sk[m]);
+                smax = max(smax, sk[m]);
+            }
+            smin = warp_min(smin);
+            smax = warp_max(smax);
+            const Bins bin(smin, smax);
+            if (smin == smax) {
+                lo = smin;
+            } else if (bin.ok) {
+                clear_hist(hist, lane);
+#pragma unroll
+                for (int m = 0; m < kSample / 32; ++m) atomicAdd(&hist[bin(sk[m])], 1u);
+                __syncwarp();
+                int dummy = 0;
+                const uint32_t b = (uint32_t)find_digit_from_top(hist, r_lo + 1, lane, &dummy);
+                // the smallest sample in bins >= b: at least r_lo + 1 samples reach it
+                uint32_t m_lo = 0xffffffffu;
+#pragma unroll
+                for (int m = 0; m < kSample / 32; ++m)
+                    if (bin(sk[m]) >= b) m_lo = min(m_lo, sk[m]);
+                lo = warp_min(m_lo);
+            }
+        }
+
+        // ---- 2. streaming pass: keys >= lo, with indices, in index order ----
+        // For lo > 0 (the key of a number) the test key >= lo is the float test
+        // v >= value(lo): NaN fails both, and -0 / +0 compare equal in both.
+        const bool keep_all = lo == 0u;
+        const float lo_f = keep_all ? 0.f : key_value(lo);
+        int nc = 0;
+        uint32_t cmax = 0u, cmin = 0xffffffffu;
+        for (int base = 0; base < n; base += kChunk) {
+            if (base > 0) load_chunk(base);
+#pragma unroll
+            for (int u = 0; u < kChunk / 128; ++u) {
                 const int e = base + 128 * u + 4 * lane;
                 const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-                uint32_t kk[4];
+                bool in[4];
                 int cnt = 0;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    kk[c] = order_key(f[c]);
                     // past the end (the row's padding) never counts
-                    if (e + c < n && kk[c] >= lo) ++cnt;
+                    in[c] = e + c < n && (keep_all || f[c] >= lo_f);
+                    cnt += in[c];
                 }
                 const uint32_t b0 = __ballot_sync(0xffffffffu, cnt & 1);
                 const uint32_t b1 = __ballot_sync(0xffffffffu, cnt & 2);
@@ -219,14 +319,15 @@ __global__ void __launch_bounds__(32 * kWarps) topk_kernel(const TopkParams P, i
                 int pos = nc + __popc(b0 & lt_mask) + 2 * __popc(b1 & lt_mask) + 4 * __popc(b2 & lt_mask);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    if (e + c < n && kk[c] >= lo) {
+                    if (in[c]) {
+                        const uint32_t kk = order_key(f[c]);
                         if (pos < cap) {
-                            ckey[pos] = kk[c];
+                            ckey[pos] = kk;
                             cidx[pos] = e + c;
                         }
                         ++pos;
-                        cmax = max(cmax, kk[c]);
-                        cmin = min(cmin, kk[c]);
+                        cmax = max(cmax, kk);
+                        cmin = min(cmin, kk);
                     }
                 }
                 nc += __popc(b0) + 2 * __popc(b1) + 4 * __popc(b2);
@@ -236,9 +337,11 @@ __global__ void __launch_bounds__(32 * kWarps) topk_kernel(const TopkParams P, i
 
         // ---- 3. exact selection ----
         if (nc >= k && nc <= cap) {
-            int need = 0;
-            const uint32_t tau = radix_rank([&](int c) { return ckey[c]; }, nc, k - 1, warp_min(cmin),
-                                            warp_max(cmax), hist, lane, &need);
+            const uint32_t kmin = warp_min(cmin), kmax = warp_max(cmax);
+            int need = k;
+            uint32_t tau = kmax;            // all candidates equal: the first k
+            if (kmin != kmax && !bin_select(ckey, nc, k, kmin, kmax, hist, lane, &tau, &need))
+                tau = radix_rank([&](int c) { return ckey[c]; }, nc, k - 1, kmin, kmax, hist, lane, &need);
             int out = 0, eq_seen = 0;
             for (int cb = 0; cb < nc && out < k; cb += 32) {
                 const int c = cb + lane;
@@ -297,8 +400,7 @@ int topk_capacity(int n, int k)
 size_t topk_smem_bytes(int n, int k)
 {
     const int cap = topk_capacity(n, k);
-    const int region = std::max(2 * cap, kSample);
-    return sizeof(uint32_t) * (size_t)kWarps * (NB + (size_t)region);
+    return sizeof(uint32_t) * (size_t)kWarps * (NB + 2 * (size_t)cap);
 }
 
 }  // namespace
