@@ -12,15 +12,16 @@
 //
 // Design (one CTA per SM, persistent, units in head-major order so the CTAs
 // in flight share one head's K/V in L2):
-//   warp 8      TMA producer: Q tile (double-buffered) and a 4-stage ring of
-//               32 KB K/V tiles, loaded in exactly the order the MMA warp
-//               consumes them: K0, K1, V0, K2, V1, ..., V(n-1).  Each tile is
-//               two 128-row x 128-byte boxes with the 128-byte swizzle.
-//   warp 9      allocates TMEM; one thread issues the MMAs.  Kept tile j goes
-//               to softmax group g = j & 1: S(j) = Q K(j)^T into S buffer g,
-//               then O(g) += P(j) V(j) with P read from TMEM, and S(j+2) is
-//               issued right behind P(j) V(j) into the same buffer (the
-//               tensor pipe runs one thread's MMAs in issue order).
+//   warp 8      TMA producer: the Q tile and a 5-stage ring of 32 KB K/V
+//               tiles, loaded in exactly the order the MMA warp consumes
+//               them: K0, K1, V0, K2, V1, ..., V(n-1).  Each tile is two
+//               128-row x 128-byte boxes with the 128-byte swizzle.
+//   warp 9      allocates TMEM and issues the MMAs (the warp runs the loop,
+//               one elected lane issues).  Kept tile j goes to softmax group
+//               g = j & 1: S(j) = Q K(j)^T into S buffer g, then
+//               O(g) += P(j) V(j) with P read from TMEM, and S(j+2) is issued
+//               right behind P(j) V(j) into the same buffer (the tensor pipe
+//               runs one thread's MMAs in issue order).
 //   warps 0-7   two softmax groups of four warps; warp % 4 is the TMEM lane
 //               quarter (thread = query row).  Each group takes every other
 //               kept tile, so the two groups run half a tile apart and one
@@ -46,7 +47,7 @@ namespace {
 
 constexpr int D = 128;
 constexpr int TT = 128;                   // tile rows (queries / keys)
-constexpr int NS = 4;                     // K/V ring stages
+constexpr int NS = 5;                     // K/V ring stages
 constexpr int kTileBytes = TT * D * 2;    // 32 KB
 constexpr int kBoxBytes = kTileBytes / 2; // 128 rows x 128 bytes
 constexpr int kThreads = 320;             // 10 warps: 8 softmax (two groups of 4), producer, MMA
@@ -75,9 +76,9 @@ struct TcParams {
 };
 
 struct __align__(1024) Smem {
-    uint8_t q[2][kTileBytes];
+    uint8_t q[kTileBytes];
     uint8_t kv[NS][kTileBytes];
-    uint64_t q_full[2], q_empty[2], kv_full[NS], kv_empty[NS];
+    uint64_t q_full, q_empty, kv_full[NS], kv_empty[NS];
     uint64_t s_full[2];         // S of softmax group g ready in TMEM buffer g
     uint64_t p_full[2];         // P of group g written (aliasing S buffer g)
     uint64_t pv_done[2];        // P V of group g completed
@@ -125,14 +126,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* b, uint32_t parity)
     return ok != 0;
 }
 
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* b, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(b)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+constexpr long long kShortWait = 4096;   // limits below this poll without suspending (test hook)
+
 // Bounded wait: true when the phase completed, false on timeout or abort.
+// try_wait may suspend the thread for a while inside one call, so a short
+// (test) limit polls with the non-blocking test_wait instead.
 __device__ __forceinline__ bool wait_phase(Smem& sm, uint64_t* b, uint32_t parity, uint32_t* status,
                                            long long limit)
 {
-    if (mbar_try_wait(b, parity)) return true;
+    const bool poll = limit < kShortWait;
+    if (poll ? mbar_test_wait(b, parity) : mbar_try_wait(b, parity)) return true;
     const long long t0 = clock64();
     for (;;) {
-        if (mbar_try_wait(b, parity)) return true;
+        if (poll ? mbar_test_wait(b, parity) : mbar_try_wait(b, parity)) return true;
         if (sm.abort_flag) return false;
         if (clock64() - t0 > limit) {
             record_status(status, VEDA_ERR_TIMEOUT);
@@ -178,12 +197,14 @@ __device__ __forceinline__ void tma_load(void* dst, const CUtensorMap* map, uint
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
+// The MMA helpers below are executed by all 32 lanes of the issuing warp
+// with warp-uniform operands; one lane, chosen by elect.sync, issues.
 __device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                         uint32_t accumulate)
 {
     asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "{\n\t.reg .pred p, e;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
@@ -192,16 +213,18 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
                                         uint32_t accumulate)
 {
     asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "{\n\t.reg .pred p, e;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
         "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 
 __device__ __forceinline__ void umma_commit(uint64_t* bar)
 {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-                 : "memory");
+    asm volatile(
+        "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar))
+        : "memory");
 }
 
 #define TMEM_LD32(taddr, r)                                                                                      \
@@ -337,9 +360,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     constexpr int kProducerWarp = 8, kMmaWarp = 9;
 
     if (threadIdx.x == 0) {
+        mbar_init(&sm.q_full, 1);
+        mbar_init(&sm.q_empty, 1);
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&sm.q_full[i], 1);
-            mbar_init(&sm.q_empty[i], 1);
             mbar_init(&sm.s_full[i], 1);
             mbar_init(&sm.p_full[i], 128);
             mbar_init(&sm.pv_done[i], 1);
@@ -374,10 +397,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             const int i = (int)(u % P.nq);
             const int64_t bh = u / P.nq;
             const int h = (int)(bh % P.H), b = (int)(bh / P.H);
-            const uint32_t qb = uq & 1;
-            if (uq >= 2 && !(ok = wait_phase(sm, &sm.q_empty[qb], ((uq >> 1) - 1) & 1, P.status, P.wait_limit))) break;
-            mbar_expect_tx(&sm.q_full[qb], kTileBytes);
-            load_box_pair(P, 0, sm.q[qb], &sm.q_full[qb], h, i * TT, b);
+            // the previous unit's last S has read the Q buffer
+            if (uq >= 1 && !(ok = wait_phase(sm, &sm.q_empty, (uq - 1) & 1, P.status, P.wait_limit))) break;
+            mbar_expect_tx(&sm.q_full, kTileBytes);
+            load_box_pair(P, 0, sm.q, &sm.q_full, h, i * TT, b);
             ++uq;
             auto load_kv = [&](int j, int which) -> bool {
                 const TileRef r = resolve(P, u, j);
@@ -399,25 +422,29 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         // drain: every issued load must land before the CTA can exit
         for (uint32_t k = (f > NS ? f - NS : 0); k < f; ++k)
             if (!drain_phase(&sm.kv_full[k % NS], (k / NS) & 1, P.status)) break;
-        for (uint32_t k = (uq > 2 ? uq - 2 : 0); k < uq; ++k)
-            if (!drain_phase(&sm.q_full[k & 1], (k >> 1) & 1, P.status)) break;
-    } else if (warp == kMmaWarp && lane == 0) {
+        if (uq > 0) drain_phase(&sm.q_full, (uq - 1) & 1, P.status);
+    } else if (warp == kMmaWarp) {
         // ------------------------------------------------- MMA issuer ---
-        // Kept tile j goes to softmax group g = j & 1.  S(j+2) reuses group g's
-        // TMEM buffer, which holds P(j): it is issued right after P(j) V(j), and
-        // the tensor pipe runs one thread's MMAs in issue order.
+        // The whole warp runs this loop (warp-uniform waits and operands); one
+        // elected lane issues each MMA and commit.  Kept tile j goes to softmax
+        // group g = j & 1.  S(j+2) reuses group g's TMEM buffer, which holds
+        // P(j): it is issued right after P(j) V(j), and the tensor pipe runs one
+        // thread's MMAs in issue order.
         constexpr uint32_t idS = idesc_bf16(false), idPV = idesc_bf16(true);
-        uint32_t uq = 0, f = 0, pc0 = 0, pc1 = 0, units_done = 0;
+        uint32_t uq = 0, pc0 = 0, pc1 = 0, units_done = 0;
+        uint32_t kst = 0, kph = 0;      // K/V ring: stage of the next tile consumed, and its fill phase
+        auto ring_next = [&]() {
+            if (++kst == NS) { kst = 0; kph ^= 1u; }
+        };
         bool ok = true;
         for (int64_t u = blockIdx.x; u < P.units && ok; u += gridDim.x) {
-            const uint32_t qb = uq & 1;
-            if (!(ok = wait_phase(sm, &sm.q_full[qb], (uq >> 1) & 1, P.status, P.wait_limit))) break;
+            if (!(ok = warp_wait(sm, &sm.q_full, uq & 1, P.status, P.wait_limit))) break;
             ++uq;
             tc_fence_after();
-            const uint32_t qaddr = smem_u32(sm.q[qb]);
+            const uint32_t qaddr = smem_u32(sm.q);
             auto issue_s = [&](int j) -> bool {
-                const uint32_t st = f % NS, g = j & 1;
-                if (!wait_phase(sm, &sm.kv_full[st], (f / NS) & 1, P.status, P.wait_limit)) return false;
+                const uint32_t st = kst, g = j & 1;
+                if (!warp_wait(sm, &sm.kv_full[st], kph, P.status, P.wait_limit)) return false;
                 tc_fence_after();
                 const uint32_t kaddr = smem_u32(sm.kv[st]);
 #pragma unroll
@@ -428,17 +455,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 }
                 umma_commit(&sm.s_full[g]);
                 umma_commit(&sm.kv_empty[st]);
-                if (j == n_list - 1) umma_commit(&sm.q_empty[qb]);   // last read of this Q tile
-                ++f;
+                if (j == n_list - 1) umma_commit(&sm.q_empty);   // last read of this Q tile
+                ring_next();
                 return true;
             };
             if (!(ok = issue_s(0))) break;
             if (n_list > 1 && !(ok = issue_s(1))) break;
             for (int j = 0; j < n_list && ok; ++j) {
-                const uint32_t g = j & 1, st = f % NS;
-                if (!(ok = wait_phase(sm, &sm.kv_full[st], (f / NS) & 1, P.status, P.wait_limit))) break;
-                if (!(ok = wait_phase(sm, &sm.p_full[g], (g ? pc1 : pc0) & 1, P.status, P.wait_limit))) break;
-                if (j == 0 && units_done > 0 && !(ok = wait_phase(sm, &sm.o_free, (units_done - 1) & 1, P.status, P.wait_limit)))
+                const uint32_t g = j & 1, st = kst;
+                if (!(ok = warp_wait(sm, &sm.kv_full[st], kph, P.status, P.wait_limit))) break;
+                if (!(ok = warp_wait(sm, &sm.p_full[g], (g ? pc1 : pc0) & 1, P.status, P.wait_limit))) break;
+                if (j == 0 && units_done > 0 &&
+                    !(ok = warp_wait(sm, &sm.o_free, (units_done - 1) & 1, P.status, P.wait_limit)))
                     break;
                 tc_fence_after();
                 const uint32_t vaddr = smem_u32(sm.kv[st]);
@@ -448,7 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                             idPV, (j >= 2 || kk > 0) ? 1u : 0u);
                 umma_commit(&sm.pv_done[g]);
                 umma_commit(&sm.kv_empty[st]);
-                ++f;
+                ring_next();
                 if (g) ++pc1; else ++pc0;
                 if (j + 2 < n_list && !(ok = issue_s(j + 2))) break;
             }
