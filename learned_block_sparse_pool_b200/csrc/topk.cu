@@ -278,8 +278,12 @@ __global__ void __launch_bounds__(32 * kWarps, 4) topk_kernel(const TopkParams P
                 lo = smin;
             } else if (bin.ok) {
                 clear_hist(hist, lane);
+                uint32_t sbin[kSample / 32];
 #pragma unroll
-                for (int m = 0; m < kSample / 32; ++m) atomicAdd(&hist[bin(sk[m])], 1u);
+                for (int m = 0; m < kSample / 32; ++m) {
+                    sbin[m] = bin(sk[m]);
+                    atomicAdd(&hist[sbin[m]], 1u);
+                }
                 __syncwarp();
                 int dummy = 0;
                 const uint32_t b = (uint32_t)find_digit_from_top(hist, r_lo + 1, lane, &dummy);
@@ -287,30 +291,33 @@ __global__ void __launch_bounds__(32 * kWarps, 4) topk_kernel(const TopkParams P
                 uint32_t m_lo = 0xffffffffu;
 #pragma unroll
                 for (int m = 0; m < kSample / 32; ++m)
-                    if (bin(sk[m]) >= b) m_lo = min(m_lo, sk[m]);
+                    if (sbin[m] >= b) m_lo = min(m_lo, sk[m]);
                 lo = warp_min(m_lo);
             }
         }
 
-        // ---- 2. streaming pass: keys >= lo, with indices, in index order ----
+        // ---- 2. streaming pass: scores >= value(lo), with indices, in index order ----
         // For lo > 0 (the key of a number) the test key >= lo is the float test
         // v >= value(lo): NaN fails both, and -0 / +0 compare equal in both.
+        // The scores are kept as they are; their keys are formed afterwards,
+        // for the kept ones only.
         const bool keep_all = lo == 0u;
         const float lo_f = keep_all ? 0.f : key_value(lo);
         int nc = 0;
-        uint32_t cmax = 0u, cmin = 0xffffffffu;
         for (int base = 0; base < n; base += kChunk) {
             if (base > 0) load_chunk(base);
+            const bool full = base + kChunk <= n;               // no row end in this chunk
 #pragma unroll
             for (int u = 0; u < kChunk / 128; ++u) {
                 const int e = base + 128 * u + 4 * lane;
                 const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+                const bool room = nc + 128 <= cap;                // no list overflow in this step
                 bool in[4];
                 int cnt = 0;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     // past the end (the row's padding) never counts
-                    in[c] = e + c < n && (keep_all || f[c] >= lo_f);
+                    in[c] = (full || e + c < n) && (keep_all || f[c] >= lo_f);
                     cnt += in[c];
                 }
                 const uint32_t b0 = __ballot_sync(0xffffffffu, cnt & 1);
@@ -320,20 +327,28 @@ __global__ void __launch_bounds__(32 * kWarps, 4) topk_kernel(const TopkParams P
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     if (in[c]) {
-                        const uint32_t kk = order_key(f[c]);
-                        if (pos < cap) {
-                            ckey[pos] = kk;
+                        if (room || pos < cap) {
+                            ckey[pos] = __float_as_uint(f[c]);
                             cidx[pos] = e + c;
                         }
                         ++pos;
-                        cmax = max(cmax, kk);
-                        cmin = min(cmin, kk);
                     }
                 }
                 nc += __popc(b0) + 2 * __popc(b1) + 4 * __popc(b2);
             }
         }
         __syncwarp();
+        // keys of the kept scores, and their range
+        uint32_t cmax = 0u, cmin = 0xffffffffu;
+        if (nc <= cap) {
+            for (int c = lane; c < nc; c += 32) {
+                const uint32_t kk = order_key(__uint_as_float(ckey[c]));
+                ckey[c] = kk;
+                cmax = max(cmax, kk);
+                cmin = min(cmin, kk);
+            }
+            __syncwarp();
+        }
 
         // ---- 3. exact selection ----
         if (nc >= k && nc <= cap) {
