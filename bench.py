@@ -18,6 +18,8 @@ timed region is bracketed by barriers and the max over ranks is reported.
 from __future__ import annotations
 
 import argparse
+import atexit
+import datetime
 import json
 import os
 import statistics
@@ -40,8 +42,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
-    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["veda", "reference"], default="veda")
     ap.add_argument("--workload", default="t2v_5.17s", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--budget", type=int, default=0, help="override the video budget")
@@ -51,6 +53,13 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ncu", action="store_true", help="short run for profiler captures (no extras)")
     return ap.parse_args()
+
+
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the
+# attention kernel in its current form, from one ncu capture of 8 of the 32
+# heads of t2v_5.17s (1.5584 GB), scaled by the units processed (x4) to the
+# full launch.  Other workloads have no capture: null.
+ATTN_TRAFFIC = {("t2v_5.17s", 32, 98): 1.5584e9 * 4}
 
 
 def peaks():
@@ -67,9 +76,12 @@ def peaks():
 # ---------------------------------------------------------------------------
 
 class ClockSampler:
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    """nvidia-smi samples every 100 ms, started before the warm-up so that it
+    is running when the timed region begins; only the samples whose
+    timestamps fall inside the timed region (wall clock) are summarised."""
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device_index: int):
         self.proc = None
@@ -81,40 +93,46 @@ class ClockSampler:
             self.ident = None
 
     def start(self):
-        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
         if self.ident:
             cmd += ["-i", self.ident]
         try:
             self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+            return
+        proc = self.proc
+        atexit.register(lambda: proc.poll() is None and proc.kill())   # no sampler outlives the run
 
-    def stop(self):
+    def stop(self, t0: float, t1: float):
+        """Summary of the samples taken between wall-clock times t0 and t1."""
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        time.sleep(0.25)
+        time.sleep(0.15)
         self.proc.terminate()
         try:
             out, _ = self.proc.communicate(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
             out, _ = self.proc.communicate()
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        rows = []
         for line in out.strip().splitlines():
             parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 8:
+            if len(parts) < 9:
                 continue
             try:
-                sm.append(float(parts[0]))
-                mx.append(float(parts[1]))
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(parts[1]), float(parts[2]), parts[5:9]))
             except ValueError:
                 continue
-            for nm, val in zip(names, parts[4:8]):
-                if val.lower().startswith("active"):
-                    reasons.add(nm)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        inside = [r for r in rows if t0 <= r[0] <= t1]
+        if not inside and rows:   # a region shorter than the sampling period: the nearest sample
+            inside = [min(rows, key=lambda r: abs(r[0] - 0.5 * (t0 + t1)))]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({nm for r in inside for nm, val in zip(names, r[3]) if val.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[1] for r in inside) if inside else None,
+                "sm_max_mhz": max(r[2] for r in inside) if inside else None,
+                "reasons": reasons, "samples": len(inside)}
 
 
 # ---------------------------------------------------------------------------
@@ -221,6 +239,8 @@ def main():
     def events():
         return [torch.cuda.Event(enable_timing=True) for _ in range(5)]
 
+    clocks = ClockSampler(local)
+    clocks.start()
     for _ in range(args.warmup):
         ev = events()
         ev[0].record(stream)
@@ -231,11 +251,10 @@ def main():
 
     evs = [events() for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(local)
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    clocks.start()
+    wall0 = time.time()
     t_start.record(stream)
     for k in range(args.steps):
         evs[k][0].record(stream)
@@ -244,7 +263,8 @@ def main():
     torch.cuda.synchronize(dev)
     if dist is not None:
         dist.barrier()
-    clk = clocks.stop()
+    wall1 = time.time()
+    clk = clocks.stop(wall0, wall1)
     st = veda.check_status(ws, stream)
     if st != 0:
         raise RuntimeError(f"device status after timing: {veda.status_string(st)}")
@@ -264,9 +284,10 @@ def main():
     esz = 2 if w.dtype == "bf16" else 4
     pool_bytes = (2 * w.n_video + w.n_ref) * w.B * w.H * w.d * esz
     rows = w.B * w.H * w.n_q_tiles
-    topk_bytes = rows * (w.n_q_tiles * 4 + w.budget_video * 4)
+    # a row's scores are read unless every tile is kept; the kept indices are written
+    topk_bytes = rows * ((w.n_q_tiles * 4 if w.budget_video < w.n_q_tiles else 0) + w.budget_video * 4)
     if w.ref_frames:
-        topk_bytes += rows * (w.n_ref_tiles * 4 + w.budget_ref * 4)
+        topk_bytes += rows * ((w.n_ref_tiles * 4 if w.budget_ref < w.n_ref_tiles else 0) + w.budget_ref * 4)
     launches_per_step = 4 + (2 if w.ref_frames else 0)
 
     res = {
@@ -293,7 +314,8 @@ def main():
         "roofline": {
             "kernel": "block-sparse attention",
             "bound": "tensor", "achieved": round(achieved_tf, 2), "peak": peak_tf, "unit": "TFLOP/s",
-            "frac": round(achieved_tf / peak_tf, 4), "traffic": None,
+            "frac": round(achieved_tf / peak_tf, 4),
+            "traffic": ATTN_TRAFFIC.get((w.name, w.H, w.budget_video)),
             "peak_kind": f"bf16 dense, sustained ({pk_src})",
             "frac_of_burst_peak": round(achieved_tf / burst_tf, 4),
             "algorithmic": f"{flops:.4g} FLOP per launch = 4*T*T*d x kept (b,h,q-tile,k-tile) pairs",
