@@ -225,16 +225,17 @@ __host__ __device__ __forceinline__ int bracket_rank(int n, int k)
 }
 
 // One warp per row.  Per-warp shared memory: histogram | candidate keys
-// (cap) | candidate indices (cap).
+// (cap + 1) | candidate indices (cap + 1); entry cap is a spare slot that
+// absorbs the stores of entries not kept.
 __global__ void __launch_bounds__(32 * kWarps, 4) topk_kernel(const TopkParams P, int cap, int r_lo)
 {
     extern __shared__ uint32_t smem[];
     const int lane = threadIdx.x & 31;
     const int w = threadIdx.x >> 5;
     const int n = P.n, k = P.k;
-    uint32_t* hist = smem + (size_t)w * (NB + 2 * cap);
+    uint32_t* hist = smem + (size_t)w * (NB + 2 * (cap + 1));
     uint32_t* ckey = hist + NB;
-    int32_t* cidx = reinterpret_cast<int32_t*>(ckey + cap);
+    int32_t* cidx = reinterpret_cast<int32_t*>(ckey + cap + 1);
     const uint32_t lt_mask = (1u << lane) - 1u;
     const bool sampled = n > kSample && r_lo < kSample - 1;
 
@@ -311,7 +312,6 @@ __global__ void __launch_bounds__(32 * kWarps, 4) topk_kernel(const TopkParams P
             for (int u = 0; u < kChunk / 128; ++u) {
                 const int e = base + 128 * u + 4 * lane;
                 const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-                const bool room = nc + 128 <= cap;                // no list overflow in this step
                 bool in[4];
                 int cnt = 0;
 #pragma unroll
@@ -324,15 +324,14 @@ __global__ void __launch_bounds__(32 * kWarps, 4) topk_kernel(const TopkParams P
                 const uint32_t b1 = __ballot_sync(0xffffffffu, cnt & 2);
                 const uint32_t b2 = __ballot_sync(0xffffffffu, cnt & 4);
                 int pos = nc + __popc(b0 & lt_mask) + 2 * __popc(b1 & lt_mask) + 4 * __popc(b2 & lt_mask);
+                // branch-free: entries that are not kept, or past the list's
+                // capacity, go to the spare slot `cap`
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    if (in[c]) {
-                        if (room || pos < cap) {
-                            ckey[pos] = __float_as_uint(f[c]);
-                            cidx[pos] = e + c;
-                        }
-                        ++pos;
-                    }
+                    const int slot = in[c] ? min(pos, cap) : cap;
+                    ckey[slot] = __float_as_uint(f[c]);
+                    cidx[slot] = e + c;
+                    pos += in[c];
                 }
                 nc += __popc(b0) + 2 * __popc(b1) + 4 * __popc(b2);
             }
@@ -415,7 +414,7 @@ int topk_capacity(int n, int k)
 size_t topk_smem_bytes(int n, int k)
 {
     const int cap = topk_capacity(n, k);
-    return sizeof(uint32_t) * (size_t)kWarps * (NB + 2 * (size_t)cap);
+    return sizeof(uint32_t) * (size_t)kWarps * (NB + 2 * ((size_t)cap + 1));
 }
 
 }  // namespace
