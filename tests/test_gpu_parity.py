@@ -273,7 +273,13 @@ def sample_units(w, n_units=64, seed=0):
     return sorted(units)
 
 
-@pytest.mark.parametrize("name", FULL)
+# The competition's fixed budgets and the R2VA formats and lengths: full-size
+# selection on every row, attention on a smaller sample of units.
+VARIANTS = ["t2v_5.17s_k16", "t2v_5.17s_k32", "t2v_5.17s_k64", "r2va_5.17s_1x1", "r2va_5.17s_4x3",
+            "r2va_10.13s", "r2va_14.38s"]
+
+
+@pytest.mark.parametrize("name", FULL + VARIANTS)
 def test_full_size_workload(dev, oracle_mod, name):
     w = workloads.get(name)
     g = workloads.make_inputs(w, device=dev)
@@ -285,6 +291,6 @@ def test_full_size_workload(dev, oracle_mod, name):
     sel = oracle_mod.select_tiles(host, w.T, w.budget_video, w.budget_ref if w.ref_frames else 0)
     rep = check_selection(oracle_mod, p, ws, iv, ir, sel, name, host)
     print(f"{name}: {rep.rows} selection rows, {len(rep.tie_band)} inside the tie band")
-    units = sample_units(w)
+    units = sample_units(w, n_units=64 if name in FULL else 24)
     _, err = check_attention(oracle_mod, w, host, p, ws, sel, units, name)
     print(f"{name}: attention on {len(units)} units: max-abs {err[0]:.3g} rel-L2 {err[1]:.3g}")

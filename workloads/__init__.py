@@ -13,6 +13,12 @@ Workload shapes follow the pages:
   * 90% / 95% sparsity (tao.media article, section "Training the Selector,
     Not the Generator"); block budgets 16 / 32 / 64 (same article, section
     "How the SN120 Competition Works").
+  * R2VA at 1:1 and 4:3 and at 10.1 s and 14.4 s (veyrul.com record "Veda
+    R2VA for MiniMax-H3", third paragraph; square and 4:3 formats also in the
+    tao.media article, section "Inside the MiniMax-H3 Studio").  The pages
+    give no resolution for 1:1 and 4:3: they keep about the 1344x768 pixel
+    count at multiples of 16 pixels (1024x1024 -> 64 x 64 latent tokens,
+    1152x864 -> 54 x 72).
 
 The latent grids (31 x 48 x 84 tokens for 5.17 s, 87 x 48 x 84 for 14.38 s,
 61 x 84 x 48 for the 10.13 s portrait clip) and the value recipes below are
@@ -152,8 +158,24 @@ def _portrait() -> Workload:
                     sweep=(budget_for_sparsity(n, 0.90), n))
 
 
+def _competition_budgets() -> Tuple[Workload, ...]:
+    """t2v 5.17 s at the competition's fixed block budgets 16 / 32 / 64."""
+    base = _t2v_517()
+    return tuple(replace(base, name=f"t2v_5.17s_k{k}", budget_video=k) for k in (16, 32, 64))
+
+
+def _r2va_variants() -> Tuple[Workload, ...]:
+    """R2VA at 1:1 and 4:3 (5.17 s) and at 10.1 s / 14.4 s (16:9)."""
+    base = _r2va()
+    return (replace(base, name="r2va_5.17s_1x1", Y=64, X=64, seed=5),
+            replace(base, name="r2va_5.17s_4x3", Y=54, X=72, seed=6),
+            replace(base, name="r2va_10.13s", frames=61, seed=7),
+            replace(base, name="r2va_14.38s", frames=87, seed=8))
+
+
 WORKLOADS: Dict[str, Workload] = {w.name: w for w in
-                                  (_tiny(), _t2v_517(), _t2v_1438(), _r2va(), _portrait())}
+                                  (_tiny(), _t2v_517(), _t2v_1438(), _r2va(), _portrait())
+                                  + _competition_budgets() + _r2va_variants()}
 
 
 def get(name: str) -> Workload:
