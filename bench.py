@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ncu", action="store_true", help="short run for profiler captures (no extras)")
+    ap.add_argument("--dense-queries", type=int, default=0, metavar="ROWS",
+                    help="time veda_dense_query_attn instead: ROWS non-video query rows over every key")
     return ap.parse_args()
 
 
@@ -222,6 +224,9 @@ def main():
     g = workloads.make_inputs(w, device=dev)
     p = make_problem(veda, w, g, args.simt)
     ws = veda.workspace(p)
+    if args.dense_queries:
+        dense_query_run(args, veda, w, g, p, ws, dev, local, rank, n, dist)
+        return
     iv, ir = veda.alloc_indices(p)
     out, _ = veda.alloc_output(p)
     stream = torch.cuda.current_stream(dev)
@@ -338,6 +343,66 @@ def main():
         ms, cores, sample = oracle_sample(w, g)
         res["cpu_baseline"] = {"value": round(ms, 1), "unit": "ms", "cores": cores, "kind": "oracle",
                                "sample": sample}
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def dense_query_run(args, veda, w, g, p, ws, dev, local, rank, n, dist):
+    """Dense-query rows (text / VLM / audio / reference tokens as queries over
+    every key of the problem): one veda_dense_query_attn per step."""
+    rows = args.dense_queries
+    gen = torch.Generator(device=dev).manual_seed(1000 + w.seed)
+    q_rows = torch.randn((w.B, rows, w.H, w.d), generator=gen, device=dev, dtype=torch.float32).to(w.torch_dtype)
+    out = torch.empty_like(q_rows)
+    stream = torch.cuda.current_stream(dev)
+    clocks = ClockSampler(local)
+    clocks.start()
+    for _ in range(args.warmup):
+        veda.dense_query_attn(p, q_rows, out, None, ws, stream)
+    st = veda.check_status(ws, stream)
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {veda.status_string(st)}")
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    wall0 = time.time()
+    t0.record(stream)
+    for _ in range(args.steps):
+        veda.dense_query_attn(p, q_rows, out, None, ws, stream)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop(wall0, time.time())
+    st = veda.check_status(ws, stream)
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {veda.status_string(st)}")
+    ms, = max_over_ranks(dist, [t0.elapsed_time(t1) / args.steps], dev)
+    tiles = w.n_q_tiles + (w.n_ref_tiles if w.n_ref else 0) + w.n_dense_tiles
+    flops = 4.0 * w.T * w.T * w.d * w.B * w.H * (-(-rows // w.T)) * tiles
+    pk, pk_src = peaks()
+    peak_tf = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    burst_tf = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    achieved = flops / (ms / 1e3) / 1e12
+    res = {
+        "metric": "ms per dense-query attention call (non-video query rows over every key)",
+        "value": round(ms / n, 4), "unit": "ms", "n_gpus": n, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms, 4), "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded N(0,1) query rows; the workload's keys)",
+        "config": dict(w.describe(), **{"dense_query_rows": rows, "key_tiles_per_query_tile": tiles,
+                                        "tflop_per_call": round(flops / 1e12, 4),
+                                        "l2": "keys larger than L2 (K, V of one call exceed 126 MB each)"}),
+        "roofline": {"kernel": "attention, every key tile", "bound": "tensor", "achieved": round(achieved, 2),
+                     "peak": peak_tf, "unit": "TFLOP/s", "frac": round(achieved / peak_tf, 4), "traffic": None,
+                     "peak_kind": f"bf16 dense, sustained ({pk_src})",
+                     "frac_of_burst_peak": round(achieved / burst_tf, 4)},
+        "clocks": clk,
+        "gpu_launches": args.steps,
+    }
     if rank == 0:
         print(json.dumps(res), flush=True)
     if dist is not None:

@@ -148,6 +148,25 @@ VEDA_API veda_status veda_block_sparse_attn(const veda_problem* p, const int32_t
                                    const int32_t* idx_ref, void* out, float* lse,
                                    void* ws, size_t ws_bytes, veda_stream_t stream);
 
+/* Dense-query rows: queries that are not video tokens (text, VLM, audio or
+ * reference tokens of a joint-attention layer) attend densely to every token
+ * of every segment of the problem -- all video tiles, all reference tiles
+ * and every dense token -- with one softmax (veyrul.com, "Veda R2VA for
+ * MiniMax-H3", second paragraph: text, VLM conditioning and audio attention
+ * stay dense; only the video and reference key tiles are selected).  The
+ * problem's budgets are not used.
+ *   q_rows   [B, n_rows, H, d] device, problem dtype, d contiguous; element
+ *            strides (q_stride_*) are multiples of 16 bytes, q_rows 16-byte
+ *            aligned; n_rows in [1, 2^30]
+ *   out      [B, n_rows, H, d] problem dtype (16-byte aligned); lse
+ *            [B, H, n_rows] fp32 or NULL
+ *   ws       a workspace of this problem (only its status word is used).
+ * Errors: VEDA_ERR_INVALID_ARG for a bad pointer, stride or row count, as
+ * for the other calls; device-side errors go to the status word. */
+VEDA_API veda_status veda_dense_query_attn(const veda_problem* p, const void* q_rows, int64_t n_rows,
+                                  int64_t q_stride_b, int64_t q_stride_tok, int64_t q_stride_h,
+                                  void* out, float* lse, void* ws, size_t ws_bytes, veda_stream_t stream);
+
 /* Steps 1-4 in one call (selection, then attention on the selected tiles),
  * stream-ordered, no host synchronisation.  idx_video / idx_ref receive the
  * kept tiles as in veda_select_tiles. */

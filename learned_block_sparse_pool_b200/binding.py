@@ -29,7 +29,7 @@ VEDA_FLAG_TEST_SHORT_WAITS = 2
 
 EXPORTS = ("veda_workspace_size", "veda_workspace_init", "veda_select_tiles", "veda_block_sparse_attn",
            "veda_attn", "veda_pool_project", "veda_score_tiles", "veda_topk_tiles", "veda_workspace_view",
-           "veda_check_status", "veda_status_string", "veda_select_tiles_noalloc")
+           "veda_check_status", "veda_status_string", "veda_select_tiles_noalloc", "veda_dense_query_attn")
 
 
 class VedaError(RuntimeError):
@@ -70,6 +70,8 @@ def lib() -> ctypes.CDLL:
         L.veda_select_tiles.argtypes = [P, vp, vp, i32p, i32p, vp, sz, vp]
         L.veda_block_sparse_attn.argtypes = [P, i32p, i32p, vp, vp, vp, sz, vp]
         L.veda_attn.argtypes = [P, vp, vp, i32p, i32p, vp, vp, vp, sz, vp]
+        i64 = ctypes.c_int64
+        L.veda_dense_query_attn.argtypes = [P, vp, i64, i64, i64, i64, vp, vp, vp, sz, vp]
         L.veda_pool_project.argtypes = [P, vp, vp, vp, sz, vp]
         L.veda_score_tiles.argtypes = [P, vp, sz, vp]
         L.veda_topk_tiles.argtypes = [P, i32p, i32p, vp, sz, vp]
@@ -204,6 +206,17 @@ def select_tiles_noalloc(p: Problem, w_q, w_k, idx_v, idx_r, stream=None) -> Non
 def block_sparse_attn(p: Problem, idx_v, idx_r, out, lse, ws, stream=None) -> None:
     _check(lib().veda_block_sparse_attn(p.ref(), _ptr(idx_v), _ptr(idx_r), out.data_ptr(), _ptr(lse),
                                         ws.data_ptr(), ws.numel(), _stream(stream)), "veda_block_sparse_attn")
+
+
+def dense_query_attn(p: Problem, q_rows, out, lse, ws, stream=None) -> None:
+    """q_rows [B, n_rows, H, d] (problem dtype, device) attend to every token
+    of every segment of p; out like q_rows, lse [B, H, n_rows] fp32 or None."""
+    B, n, H, d = q_rows.shape
+    if (B, H, d) != (p.B, p.H, p.d) or q_rows.dtype != p.dtype or q_rows.stride(3) != 1:
+        raise ValueError("q_rows must be [B, n_rows, H, d] of the problem's dtype, d contiguous")
+    sb, st, sh, _ = q_rows.stride()
+    _check(lib().veda_dense_query_attn(p.ref(), q_rows.data_ptr(), n, sb, st, sh, out.data_ptr(), _ptr(lse),
+                                       ws.data_ptr(), ws.numel(), _stream(stream)), "veda_dense_query_attn")
 
 
 def attn(p: Problem, w_q, w_k, idx_v, idx_r, out, lse, ws, stream=None) -> None:

@@ -210,6 +210,7 @@ veda_status do_attn(const veda_problem& p, const Layout& L, const int32_t* idx_v
     memset(&A, 0, sizeof A);
     A.q = p.q;
     A.qsb = p.q_stride_b; A.qst = p.q_stride_tok; A.qsh = p.q_stride_h;
+    A.n_qtok = p.video.n_tokens;
     A.video = to_segment(p.video, p.tile);
     A.ref = to_segment(p.ref, p.tile);
     A.dense = to_segment(p.dense, p.tile);
@@ -220,6 +221,38 @@ veda_status do_attn(const veda_problem& p, const Layout& L, const int32_t* idx_v
     A.out = out;
     A.lse = lse;
     A.B = p.B; A.H = p.H; A.d = p.d; A.T = p.tile; A.nq = (int32_t)L.nq;
+    A.dtype = p.dtype;
+    A.scale = p.softmax_scale > 0.f ? p.softmax_scale : 1.0f / sqrtf((float)p.d);
+    A.status = at<uint32_t>(ws, 0);
+    A.short_waits = (p.flags & VEDA_FLAG_TEST_SHORT_WAITS) ? 1 : 0;
+    if (!(p.flags & VEDA_FLAG_SIMT_ATTENTION) && attn_tc_supported(A)) return from_cuda(launch_attn_tc(A, s));
+    return from_cuda(launch_attn_simt(A, s));
+}
+
+// Dense-query rows: every query row attends to every token of every segment.
+veda_status do_dense_query_attn(const veda_problem& p, const void* q_rows, int64_t n_rows, int64_t sb, int64_t st,
+                                int64_t sh, void* out, float* lse, void* ws, cudaStream_t s)
+{
+    const size_t es = esize(p.dtype);
+    if (n_rows < 1 || n_rows > (int64_t)1 << 30 || !q_rows || !aligned16(q_rows)) return VEDA_ERR_INVALID_ARG;
+    if (!stride_ok(sb, es) || !stride_ok(st, es) || !stride_ok(sh, es)) return VEDA_ERR_INVALID_ARG;
+    if (!out || !aligned16(out) || (lse && ((uintptr_t)lse & 3u))) return VEDA_ERR_INVALID_ARG;
+    AttnParams A;
+    memset(&A, 0, sizeof A);
+    A.q = q_rows;
+    A.qsb = sb; A.qst = st; A.qsh = sh;
+    A.n_qtok = n_rows;
+    A.video = to_segment(p.video, p.tile);
+    A.ref = to_segment(p.ref, p.tile);
+    A.dense = to_segment(p.dense, p.tile);
+    A.idx_v = nullptr;                  // every video tile
+    A.idx_r = nullptr;                  // every reference tile
+    A.k_v = A.video.n_tiles;
+    A.k_r = p.ref.n_tokens > 0 ? A.ref.n_tiles : 0;
+    A.out = out;
+    A.lse = lse;
+    A.B = p.B; A.H = p.H; A.d = p.d; A.T = p.tile;
+    A.nq = (int32_t)((n_rows + p.tile - 1) / p.tile);
     A.dtype = p.dtype;
     A.scale = p.softmax_scale > 0.f ? p.softmax_scale : 1.0f / sqrtf((float)p.d);
     A.status = at<uint32_t>(ws, 0);
@@ -301,6 +334,17 @@ veda_status veda_block_sparse_attn(const veda_problem* p, const int32_t* idx_vid
     if (!ws || ((uintptr_t)ws % kAlign) != 0 || ws_bytes < kAlign) return VEDA_ERR_WORKSPACE;
     const Layout L = layout(*p);
     return do_attn(*p, L, idx_video, idx_ref, out, lse, ws, (cudaStream_t)stream);
+}
+
+veda_status veda_dense_query_attn(const veda_problem* p, const void* q_rows, int64_t n_rows, int64_t q_stride_b,
+                                  int64_t q_stride_tok, int64_t q_stride_h, void* out, float* lse, void* ws,
+                                  size_t ws_bytes, veda_stream_t stream)
+{
+    veda_status st = validate(p);
+    if (st != VEDA_OK) return st;
+    if (!ws || ((uintptr_t)ws % kAlign) != 0 || ws_bytes < kAlign) return VEDA_ERR_WORKSPACE;
+    return do_dense_query_attn(*p, q_rows, n_rows, q_stride_b, q_stride_tok, q_stride_h, out, lse, ws,
+                               (cudaStream_t)stream);
 }
 
 veda_status veda_attn(const veda_problem* p, const void* w_q, const void* w_k, int32_t* idx_video,

@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(2 * TILE) attn_simt_kernel(const AttnParams P)
     const int row = tid >> 1;
     const int half = tid & 1;
     const int64_t t = (int64_t)i * TILE + row;
-    const bool valid_q = t < P.video.n;
+    const bool valid_q = t < P.n_qtok;
     const float qscale = P.scale * 1.4426950408889634f;   // logits in base-2 units
 
     float q[4 * NC], o[4 * NC];
@@ -87,10 +87,10 @@ __global__ void __launch_bounds__(2 * TILE) attn_simt_kernel(const AttnParams P)
         int tile;
         if (jt < P.k_v) {
             S = &P.video;
-            tile = P.idx_v[idx_row * P.k_v + jt];
+            tile = P.idx_v ? P.idx_v[idx_row * P.k_v + jt] : jt;
         } else if (jt < P.k_v + P.k_r) {
             S = &P.ref;
-            tile = P.idx_r[idx_row * P.k_r + (jt - P.k_v)];
+            tile = P.idx_r ? P.idx_r[idx_row * P.k_r + (jt - P.k_v)] : jt - P.k_v;
         } else {
             S = &P.dense;
             tile = jt - P.k_v - P.k_r;
@@ -166,13 +166,13 @@ __global__ void __launch_bounds__(2 * TILE) attn_simt_kernel(const AttnParams P)
 
     if (!valid_q) return;
     const float inv = 1.f / l;
-    Tin* op = static_cast<Tin*>(P.out) + (((int64_t)b * P.video.n + t) * P.H + h) * D;
+    Tin* op = static_cast<Tin*>(P.out) + (((int64_t)b * P.n_qtok + t) * P.H + h) * D;
 #pragma unroll
     for (int c = 0; c < NC; ++c)
         store4(op + 8 * c + 4 * half, make_float4(o[4 * c] * inv, o[4 * c + 1] * inv,
                                                   o[4 * c + 2] * inv, o[4 * c + 3] * inv));
     if (P.lse && half == 0)
-        P.lse[((int64_t)b * P.H + h) * P.video.n + t] = m * 0.6931471805599453f + logf(l);
+        P.lse[((int64_t)b * P.H + h) * P.n_qtok + t] = m * 0.6931471805599453f + logf(l);
 }
 
 template <typename Tin, int D, int TILE>

@@ -62,6 +62,7 @@ struct TcParams {
     CUtensorMap tm[7];          // Q, Kv, Vv, Kr, Vr, Kd, Vd
     int8_t pos_h[7], pos_n[7], pos_b[7];
     int64_t n_tok[3];           // video, ref, dense tokens
+    int64_t n_qtok;             // query tokens (rows of Q and of the output)
     int32_t n_tiles[3];
     const int32_t* idx_v;
     const int32_t* idx_r;
@@ -325,10 +326,10 @@ __device__ __forceinline__ TileRef resolve(const TcParams& P, int64_t row, int j
     TileRef r;
     if (j < P.k_v) {
         r.seg = 0;
-        r.tile = __ldg(P.idx_v + row * P.k_v + j);
+        r.tile = P.idx_v ? __ldg(P.idx_v + row * P.k_v + j) : j;   // null: every tile
     } else if (j < P.k_v + P.k_r) {
         r.seg = 1;
-        r.tile = __ldg(P.idx_r + row * P.k_r + (j - P.k_v));
+        r.tile = P.idx_r ? __ldg(P.idx_r + row * P.k_r + (j - P.k_v)) : j - P.k_v;
     } else {
         r.seg = 2;
         r.tile = j - P.k_v - P.k_r;
@@ -615,14 +616,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             const float inv = 1.f / L;
             const float c0 = f0 * inv, c1 = f1 * inv;
             const int64_t tok = (int64_t)i * TT + row;
-            __nv_bfloat16* dst = P.out + (((int64_t)b * P.n_tok[0] + tok) * P.H + h) * D + 64 * g;
+            __nv_bfloat16* dst = P.out + (((int64_t)b * P.n_qtok + tok) * P.H + h) * D + 64 * g;
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
                 uint32_t o0[32], o1[32];
                 TMEM_LD32(tmem + lane_off + col_o(0) + 64 * g + 32 * q, o0);
                 TMEM_LD32(tmem + lane_off + col_o(1) + 64 * g + 32 * q, o1);
                 tmem_wait_ld();
-                if (tok < P.n_tok[0]) {
+                if (tok < P.n_qtok) {
 #pragma unroll
                     for (int c = 0; c < 32; c += 8) {
                         float v[8];
@@ -646,8 +647,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                     }
                 }
             }
-            if (P.lse && g == 0 && tok < P.n_tok[0])
-                P.lse[((int64_t)b * P.H + h) * P.n_tok[0] + tok] = (M + __log2f(L)) * 0.69314718055994531f;
+            if (P.lse && g == 0 && tok < P.n_qtok)
+                P.lse[((int64_t)b * P.H + h) * P.n_qtok + tok] = (M + __log2f(L)) * 0.69314718055994531f;
             tc_fence_before();
             mbar_arrive(&sm.o_free);
         }
@@ -730,7 +731,7 @@ cudaError_t launch_attn_tc(const AttnParams& a, cudaStream_t s)
     if (!enc) return cudaErrorNotSupported;
     TcParams P;
     memset(&P, 0, sizeof P);
-    bool ok = make_map(enc, &P.tm[0], &P.pos_h[0], &P.pos_n[0], &P.pos_b[0], a.q, a.B, a.video.n, a.H, a.qsb,
+    bool ok = make_map(enc, &P.tm[0], &P.pos_h[0], &P.pos_n[0], &P.pos_b[0], a.q, a.B, a.n_qtok, a.H, a.qsb,
                        a.qst, a.qsh);
     const Segment* segs[3] = {&a.video, &a.ref, &a.dense};
     for (int g = 0; g < 3 && ok; ++g) {
@@ -758,6 +759,7 @@ cudaError_t launch_attn_tc(const AttnParams& a, cudaStream_t s)
     P.B = a.B;
     P.H = a.H;
     P.nq = a.nq;
+    P.n_qtok = a.n_qtok;
     P.units = units;
     P.out = static_cast<__nv_bfloat16*>(a.out);
     P.lse = a.lse;

@@ -74,12 +74,13 @@ cudaError_t launch_topk(const TopkParams& p, cudaStream_t s);
 struct AttnParams {
     const void* q;
     int64_t qsb, qst, qsh;
+    int64_t n_qtok;         // query tokens (the video's own, or dense-query rows)
     Segment video, ref, dense;
-    const int32_t* idx_v;   // [B, H, nq, k_v]
-    const int32_t* idx_r;   // [B, H, nq, k_r] or null
+    const int32_t* idx_v;   // [B, H, nq, k_v]; null: every video tile, in order (k_v = tiles)
+    const int32_t* idx_r;   // [B, H, nq, k_r]; null: every reference tile (or no reference)
     int32_t k_v, k_r;
-    void* out;              // [B, n_video, H, d]
-    float* lse;             // [B, H, n_video] or null
+    void* out;              // [B, n_qtok, H, d]
+    float* lse;             // [B, H, n_qtok] or null
     int32_t B, H, d, T, nq;
     int32_t dtype;
     float scale;            // softmax scale (natural-log units)

@@ -54,7 +54,7 @@ class _Problem(ctypes.Structure):
     _fields_ = [("q", _c_ptr), ("qsb", _c_i64), ("qst", _c_i64), ("qsh", _c_i64),
                 ("dtype", ctypes.c_int), ("B", _c_i64), ("H", _c_i64), ("d", _c_i64),
                 ("T", _c_i64), ("video", _Segment), ("ref", _Segment), ("dense", _Segment),
-                ("scale", ctypes.c_double)]
+                ("scale", ctypes.c_double), ("nq_tok", _c_i64)]
 
 
 def lib():
@@ -158,8 +158,10 @@ def attend(q: torch.Tensor, video: Tuple[torch.Tensor, torch.Tensor], T: int,
            scale: Optional[float] = None) -> Tuple[np.ndarray, np.ndarray]:
     """Restricted softmax attention for the listed (b, h, query tile) units.
 
+    q holds the query tokens: the video's own, or the rows of non-video
+    (dense) queries, which the caller pairs with every tile (`all_tiles`).
     Returns out [n_units, T, d] and lse [n_units, T] in fp64 (NaN rows past the
-    end of the video)."""
+    last query token)."""
     q = _cpu(q)
     B, N, H, d = q.shape
     keep = []
@@ -190,6 +192,7 @@ def attend(q: torch.Tensor, video: Tuple[torch.Tensor, torch.Tensor], T: int,
     p.ref = seg(ref)
     p.dense = seg(dense)
     p.scale = (1.0 / math.sqrt(d)) if scale is None else float(scale)
+    p.nq_tok = N
 
     idx_v = np.ascontiguousarray(idx_v, np.int32)
     k_v = idx_v.shape[-1]
@@ -233,3 +236,23 @@ def attend_units(inp: Dict[str, torch.Tensor], T: int, idx_v: np.ndarray,
     dense = (inp["k_dense"], inp["v_dense"]) if "k_dense" in inp else None
     return attend(inp["q"], (inp["k"], inp["v"]), T, idx_v, units, ref=ref, idx_r=idx_r,
                   dense=dense, scale=scale)
+
+
+def attend_dense_queries(inp: Dict[str, torch.Tensor], q_rows: torch.Tensor, T: int, units,
+                         scale: Optional[float] = None):
+    """Dense-query rows: q_rows [B, n_rows, H, d] (text, VLM, audio or
+    reference tokens as queries) attend to every tile of every segment of the
+    problem `inp` -- all video tiles, all reference tiles, every dense token.
+    units: (b, h, query tile of q_rows) triples.  Same outputs as attend()."""
+    B, n_rows, H, d = q_rows.shape
+    n_v = -(-inp["k"].shape[1] // T)
+    nq = -(-n_rows // T)
+    idx_v = np.ascontiguousarray(np.broadcast_to(np.arange(n_v, dtype=np.int32), (B, H, nq, n_v)))
+    ref, idx_r = None, None
+    if "k_ref" in inp:
+        n_r = -(-inp["k_ref"].shape[1] // T)
+        ref = (inp["k_ref"], inp["v_ref"])
+        idx_r = np.ascontiguousarray(np.broadcast_to(np.arange(n_r, dtype=np.int32), (B, H, nq, n_r)))
+    dense = (inp["k_dense"], inp["v_dense"]) if "k_dense" in inp else None
+    return attend(q_rows, (inp["k"], inp["v"]), T, idx_v, units, ref=ref, idx_r=idx_r, dense=dense,
+                  scale=scale)

@@ -208,13 +208,14 @@ typedef struct {
     int64_t B, H, d, T;
     oracle_segment video, ref, dense;   /* ref.n == 0 / dense.n == 0: absent */
     double scale;                       /* softmax scale applied to q.k */
+    int64_t nq_tok;                     /* query tokens: the video's own, or the rows of
+                                           non-video (dense) queries */
 } oracle_problem;
 
 /*
  * Block-sparse attention restricted to the kept tiles.
  *
- * For query token t of video query tile i (valid tokens only; queries are the
- * video tokens), the key set is
+ * For query token t of query tile i (valid tokens only), the key set is
  *     every valid token of each kept video tile   (idx_v row of (b,h,i))
  *   + every valid token of each kept reference tile (idx_r row, if present)
  *   + every dense (text / VLM / audio) token.
@@ -224,15 +225,21 @@ typedef struct {
  * Padded key slots beyond a segment's end are not keys at all (excluded),
  * the reading of the zero-padded last tile.
  *
+ * The queries are the video tokens (nq_tok = video.n), or, for dense-query
+ * rows, the tokens of a non-video segment (text, VLM, audio or reference
+ * tokens of a joint-attention layer) attending to every tile: the caller then
+ * lists every tile of every segment (veyrul.com, "Veda R2VA for MiniMax-H3",
+ * second paragraph: text, VLM and audio attention stay dense).
+ *
  * units: n_units triples (b, h, i).  out: [n_units][T][d]; lse: [n_units][T]
- * (rows of tokens past the end of the video are set to NAN).
+ * (rows of tokens past the last query token are set to NAN).
  */
 void oracle_attend(const oracle_problem* p, const int32_t* idx_v, int64_t k_v,
                    const int32_t* idx_r, int64_t k_r, const int64_t* units, int64_t n_units,
                    double* out, double* lse)
 {
     const int64_t T = p->T, d = p->d, H = p->H;
-    const int64_t nq = (p->video.n + T - 1) / T;
+    const int64_t nq = (p->nq_tok + T - 1) / T;
     const int64_t max_keys = k_v * T + (p->ref.n > 0 ? k_r * T : 0) + p->dense.n;
 
 #pragma omp parallel
@@ -274,7 +281,7 @@ void oracle_attend(const oracle_problem* p, const int32_t* idx_v, int64_t k_v,
             for (int64_t tt = 0; tt < T; ++tt) {
                 const int64_t t = i * T + tt;
                 double* o = out + (u * T + tt) * d;
-                if (t >= p->video.n) {
+                if (t >= p->nq_tok) {
                     for (int64_t e = 0; e < d; ++e) o[e] = NAN;
                     if (lse) lse[u * T + tt] = NAN;
                     continue;

@@ -184,6 +184,30 @@ def test_index_and_output_arguments_checked(L):
     assert L.veda_topk_tiles(ctypes.byref(q), 0x500000, 0x510000, ws, n, None) == B.VEDA_ERR_INVALID_ARG
 
 
+def test_dense_query_arguments_checked(L):
+    p = _problem()
+    st, n = _ws_size(L, p)
+    ws, q, out = 0x800000, 0x900000, 0xA00000
+    H, d = 4, 128
+    ok = (q, 10, 10 * H * d, H * d, d, out, None, ws, n, None)
+
+    def call(*a):
+        return L.veda_dense_query_attn(ctypes.byref(p), *a)
+    bad = [
+        (0, 10, 10 * H * d, H * d, d, out, None, ws, n, None),            # no query rows
+        (q + 8, 10, 10 * H * d, H * d, d, out, None, ws, n, None),        # misaligned rows
+        (q, 0, 10 * H * d, H * d, d, out, None, ws, n, None),             # no rows
+        (q, 10, 10 * H * d, H * d + 4, d, out, None, ws, n, None),        # stride not 16-byte
+        (q, 10, 10 * H * d, H * d, d, out + 8, None, ws, n, None),        # misaligned output
+        (q, 10, 10 * H * d, H * d, d, out, 0xB00002, ws, n, None),        # misaligned lse
+    ]
+    for a in bad:
+        assert call(*a) == B.VEDA_ERR_INVALID_ARG, a
+    assert call(q, 10, 10 * H * d, H * d, d, out, None, None, n, None) == B.VEDA_ERR_WORKSPACE
+    q_bad = _problem(d=96)
+    assert L.veda_dense_query_attn(ctypes.byref(q_bad), *ok) == B.VEDA_ERR_UNSUPPORTED
+
+
 def test_workspace_view_bounds(L):
     p = _problem(**{"ref.n_tokens": 0, "ref.budget": 0})
     st, n = _ws_size(L, p)

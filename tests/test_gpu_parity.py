@@ -204,6 +204,56 @@ def test_batch_two_non_packed_strides(dev, oracle_mod):
     check_attention(oracle_mod, w, inp, p, ws, sel, units, "batch2")
 
 
+def check_dense_queries(oracle_mod, w, inp, p, ws, q_rows, units, what):
+    """veda_dense_query_attn against the oracle's dense-query rows."""
+    B, n, H, d = q_rows.shape
+    out = torch.full((B, n, H, d), float("nan"), dtype=p.dtype, device=p.device)
+    lse = torch.full((B, H, n), float("nan"), dtype=torch.float32, device=p.device)
+    veda.dense_query_attn(p, q_rows.to(p.device), out, lse, ws)
+    assert veda.check_status(ws) == 0
+    want, want_lse = oracle_mod.attend_dense_queries(inp, q_rows, w.T, units)
+    err = assert_close(gather_units(out, units, w.T), want, p.dtype, what)
+    got_lse = gather_lse(lse, units, w.T)
+    m = ~np.isnan(want_lse)
+    assert np.abs(got_lse[m] - want_lse[m]).max() < (1e-4 if p.dtype == torch.float32 else 2e-2)
+    return err
+
+
+def _query_rows(w, n_rows, seed):
+    gen = torch.Generator().manual_seed(seed)
+    return torch.randn(w.B, n_rows, w.H, w.d, generator=gen).to(w.torch_dtype)
+
+
+@pytest.mark.parametrize("simt", [False, True], ids=["default", "simt"])
+@pytest.mark.parametrize("name,n_rows", [("t2v_ragged", 200), ("r2va_ragged", 300), ("tiny", 128)])
+def test_dense_query_rows(dev, oracle_mod, name, n_rows, simt):
+    """Text / VLM / audio / reference-token queries attending to every tile of
+    every segment (ragged query rows; a reference segment in the r2va case)."""
+    w = workloads.get("tiny") if name == "tiny" else REDUCED[name]()
+    inp = workloads.make_inputs(w)
+    g = to_dev(inp, dev)
+    p = make_problem(w, g, flags=veda.binding.VEDA_FLAG_SIMT_ATTENTION if simt else 0)
+    ws = veda.workspace(p)
+    q_rows = _query_rows(w, n_rows, 21)
+    units = [(b, h, i) for b in range(w.B) for h in range(w.H) for i in range(-(-n_rows // w.T))]
+    check_dense_queries(oracle_mod, w, inp, p, ws, q_rows, units, f"{name} dense queries")
+
+
+def test_dense_query_rows_full_size(dev, oracle_mod):
+    """The text and audio tokens of t2v 5.17 s (768 rows) as queries over all
+    124,992 video and 768 dense keys, on sampled units."""
+    w = workloads.get("t2v_5.17s")
+    g = workloads.make_inputs(w, device=dev)
+    p = make_problem(w, g)
+    ws = veda.workspace(p)
+    q_rows = _query_rows(w, w.n_dense, 22)
+    host = {k: v.cpu() for k, v in g.items()}
+    nq = -(-w.n_dense // w.T)
+    units = [(0, 0, 0), (0, w.H - 1, nq - 1), (0, 7, 2), (0, 19, 4)]
+    err = check_dense_queries(oracle_mod, w, host, p, ws, q_rows, units, "t2v_5.17s dense queries")
+    print(f"t2v_5.17s dense queries: {len(units)} units: max-abs {err[0]:.3g} rel-L2 {err[1]:.3g}")
+
+
 @pytest.mark.parametrize("simt", [False, True], ids=["default", "simt"])
 def test_out_of_range_index_is_flagged(dev, simt):
     w = _reduced("t2v_5.17s")

@@ -34,6 +34,8 @@ MUTANTS = {
                                      "dot += qrow[e] * elem(s->v, p->dtype, base + e);"),
     "attend_no_max_subtraction": ("const double w = exp(logit[a] - mx);", "const double w = exp(logit[a]);"),
     "attend_unnormalised": ("for (int64_t e = 0; e < d; ++e) o[e] = o[e] / z;", ""),
+    "attend_query_tiles_from_video_length": ("const int64_t nq = (p->nq_tok + T - 1) / T;",
+                                             "const int64_t nq = (p->video.n + T - 1) / T;"),
 }
 
 

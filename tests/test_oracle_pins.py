@@ -338,6 +338,30 @@ def test_attend_masked_dense_equivalence_with_reference_segment(oracle_mod):
         np.testing.assert_allclose(out[u, :c], want, rtol=1e-11, atol=1e-12)
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_dense_query_rows_are_dense_attention(oracle_mod, dtype):
+    """Non-video query rows attending to every tile (reference present, ragged
+    query, video, reference and dense tails) equal textbook dense attention
+    over the concatenated keys."""
+    B, H, d, T = 2, 2, 16, 8
+    N, Nr, Nd, Nq = 29, 13, 6, 21
+    p = _problem(5, B, H, d, T, N, n_ref=Nr, n_dense=Nd, dtype=dtype)
+    gen = torch.Generator().manual_seed(55)
+    q_rows = torch.randn(B, Nq, H, d, generator=gen).to(dtype)
+    nq = -(-Nq // T)
+    units = [(b, h, i) for b in range(B) for h in range(H) for i in range(nq)]
+    out, lse = oracle_mod.attend_dense_queries(p, q_rows, T, units, scale=0.4)
+    for u, (b, h, i) in enumerate(units):
+        qs = q_rows[b, i * T:min(Nq, (i + 1) * T), h].double()
+        keys = torch.cat([p["k"][b, :, h], p["k_ref"][b, :, h], p["k_dense"][b, :, h]]).double()
+        vals = torch.cat([p["v"][b, :, h], p["v_ref"][b, :, h], p["v_dense"][b, :, h]]).double()
+        c = qs.shape[0]
+        np.testing.assert_allclose(out[u, :c], _sdpa(qs, keys, vals, scale=0.4).numpy(), rtol=1e-11, atol=1e-12)
+        assert np.isnan(out[u, c:]).all()
+        want_lse = torch.logsumexp((qs @ keys.T) * 0.4, dim=1).numpy()
+        np.testing.assert_allclose(lse[u, :c], want_lse, rtol=1e-12, atol=1e-12)
+
+
 def test_attend_all_ones_values(oracle_mod):
     """Softmax weights sum to one: with V = 1 every output is exactly 1."""
     B, H, d, T, N, Nd = 1, 2, 8, 4, 23, 5
