@@ -70,7 +70,9 @@ typedef enum {
     VEDA_ERR_WORKSPACE = -3,    /* workspace NULL, misaligned or too small             */
     VEDA_ERR_CUDA = -4,         /* a CUDA launch or driver call failed                 */
     VEDA_ERR_TIMEOUT = -5,      /* device: a bounded wait ran out (kernel returned)    */
-    VEDA_ERR_BAD_INDEX = -6     /* device: a kept-tile index was outside its segment   */
+    VEDA_ERR_BAD_INDEX = -6,    /* device: a kept-tile index was outside its segment   */
+    VEDA_ERR_FORMAT = -7,       /* a selector artifact is malformed or off its layout  */
+    VEDA_ERR_IO = -8            /* a selector artifact could not be opened or read     */
 } veda_status;
 
 typedef enum { VEDA_F32 = 0, VEDA_BF16 = 1 } veda_dtype;
@@ -222,6 +224,49 @@ VEDA_API veda_status veda_check_status(void* ws, veda_stream_t stream);
 
 /* Static, human-readable name of a status code. */
 VEDA_API const char* veda_status_string(veda_status s);
+
+/* ---- selector artifacts --------------------------------------------------
+ * The trained selector projections ship as a safetensors file: the published
+ * competition artifact holds exactly 100 float16 tensors, the query and key
+ * projections of 50 layers, each of shape (56, 384, 128), in at most
+ * 560,000,000 bytes, with metadata that names the miner's hotkey
+ * (tao.media, "Affine launches MiniMax-H3 video studio...", section "How the
+ * SN120 Competition Works").  The R2VA predictor is stored in FP8 and
+ * dequantised to BF16 at load (veyrul.com, "Veda R2VA for MiniMax-H3",
+ * second paragraph); no scale format is published, so FP8 (E4M3) tensors are
+ * read with a caller-given scale.  A tensor of shape (H, d, r) is the
+ * [H, d, r] weight layout that veda_select_tiles takes.
+ * All of this is host code: the caller copies converted tensors to the
+ * device.  The reader owns its memory until veda_selector_close. */
+typedef struct veda_selector veda_selector;
+
+/* Read and check a safetensors file: header length, JSON header, dtypes
+ * (F16, BF16, F32, F8_E4M3), shapes, and byte ranges that tile the data
+ * section exactly.  VEDA_ERR_IO: cannot be read; VEDA_ERR_FORMAT: malformed. */
+VEDA_API veda_status veda_selector_open(const char* path, veda_selector** out);
+VEDA_API void veda_selector_close(veda_selector* s);
+
+/* Check the published layout: exactly n_tensors tensors, each F16 or
+ * F8_E4M3 with shape shape[0..ndim), the file at most max_file_bytes
+ * (<= 0: no limit), and (if required_meta_key is not NULL) a non-empty
+ * metadata value under that key.  VEDA_ERR_FORMAT when anything differs. */
+VEDA_API veda_status veda_selector_check(const veda_selector* s, int32_t n_tensors, const int64_t* shape,
+                                int32_t ndim, int64_t max_file_bytes, const char* required_meta_key);
+
+/* Tensors are indexed 0..count-1 in data-section order. */
+VEDA_API int32_t veda_selector_count(const veda_selector* s);
+VEDA_API veda_status veda_selector_find(const veda_selector* s, const char* name, int32_t* index);
+/* name / dtype point into the reader (valid until close); shape receives ndim
+ * (<= 8) extents.  Any output pointer may be NULL. */
+VEDA_API veda_status veda_selector_info(const veda_selector* s, int32_t index, const char** name,
+                               const char** dtype, int32_t* ndim, int64_t* shape);
+/* The metadata value under `key`, or NULL. */
+VEDA_API const char* veda_selector_metadata(const veda_selector* s, const char* key);
+/* Tensor `index`, times `scale` (> 0; 1 for F16 / BF16 / F32 data), into host
+ * `dst` as fp32 or bf16 (round to nearest, ties to even), row-major in the
+ * stored shape.  dst_bytes must hold every element. */
+VEDA_API veda_status veda_selector_read(const veda_selector* s, int32_t index, veda_dtype out_dtype, float scale,
+                               void* dst, size_t dst_bytes);
 
 #ifdef __cplusplus
 }

@@ -23,13 +23,17 @@ VEDA_ERR_WORKSPACE = -3
 VEDA_ERR_CUDA = -4
 VEDA_ERR_TIMEOUT = -5
 VEDA_ERR_BAD_INDEX = -6
+VEDA_ERR_FORMAT = -7
+VEDA_ERR_IO = -8
 VEDA_F32, VEDA_BF16 = 0, 1
 VEDA_FLAG_SIMT_ATTENTION = 1
 VEDA_FLAG_TEST_SHORT_WAITS = 2
 
 EXPORTS = ("veda_workspace_size", "veda_workspace_init", "veda_select_tiles", "veda_block_sparse_attn",
            "veda_attn", "veda_pool_project", "veda_score_tiles", "veda_topk_tiles", "veda_workspace_view",
-           "veda_check_status", "veda_status_string", "veda_select_tiles_noalloc", "veda_dense_query_attn")
+           "veda_check_status", "veda_status_string", "veda_select_tiles_noalloc", "veda_dense_query_attn",
+           "veda_selector_open", "veda_selector_close", "veda_selector_check", "veda_selector_count",
+           "veda_selector_find", "veda_selector_info", "veda_selector_metadata", "veda_selector_read")
 
 
 class VedaError(RuntimeError):
@@ -81,9 +85,22 @@ def lib() -> ctypes.CDLL:
         L.veda_select_tiles_noalloc.argtypes = [P, vp, vp, i32p, i32p, vp]
         L.veda_status_string.argtypes = [ctypes.c_int]
         L.veda_status_string.restype = ctypes.c_char_p
+        L.veda_selector_open.argtypes = [ctypes.c_char_p, ctypes.POINTER(vp)]
+        L.veda_selector_close.argtypes = [vp]
+        L.veda_selector_check.argtypes = [vp, ctypes.c_int32, ctypes.POINTER(ctypes.c_int64), ctypes.c_int32,
+                                          ctypes.c_int64, ctypes.c_char_p]
+        L.veda_selector_count.argtypes = [vp]
+        L.veda_selector_find.argtypes = [vp, ctypes.c_char_p, ctypes.POINTER(ctypes.c_int32)]
+        L.veda_selector_info.argtypes = [vp, ctypes.c_int32, ctypes.POINTER(ctypes.c_char_p),
+                                         ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_int32),
+                                         ctypes.POINTER(ctypes.c_int64)]
+        L.veda_selector_metadata.argtypes = [vp, ctypes.c_char_p]
+        L.veda_selector_read.argtypes = [vp, ctypes.c_int32, ctypes.c_int, ctypes.c_float, vp, sz]
         for name in EXPORTS:
-            if name != "veda_status_string":
+            if name not in ("veda_status_string", "veda_selector_close", "veda_selector_metadata"):
                 getattr(L, name).restype = ctypes.c_int
+        L.veda_selector_close.restype = None
+        L.veda_selector_metadata.restype = ctypes.c_char_p
         _lib = L
     return _lib
 
@@ -254,3 +271,79 @@ def workspace_view(p: Problem, ws, which: int) -> torch.Tensor:
 def check_status(ws, stream=None) -> int:
     """Synchronise the stream and return (and clear) the sticky device status."""
     return lib().veda_check_status(ws.data_ptr(), _stream(stream))
+
+
+# ---------------------------------------------------------------------------
+# selector artifacts (host)
+# ---------------------------------------------------------------------------
+
+# The published competition layout: 100 float16 tensors (Q and K projections
+# of 50 layers), each (56, 384, 128), at most 560,000,000 bytes.
+PUBLISHED_LAYOUT = {"n_tensors": 100, "shape": (56, 384, 128), "max_file_bytes": 560_000_000}
+
+
+class Selector:
+    """A selector artifact read by libveda: names, dtypes, shapes, metadata, and
+    tensors converted to fp32 or bf16 (host torch tensors)."""
+
+    def __init__(self, path: str):
+        h = ctypes.c_void_p()
+        _check(lib().veda_selector_open(os.fsencode(path), ctypes.byref(h)), "veda_selector_open")
+        self._h = h
+
+    def close(self) -> None:
+        if self._h:
+            lib().veda_selector_close(self._h)
+            self._h = None
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def check(self, n_tensors: int, shape, max_file_bytes: int = 0, required_meta_key: Optional[str] = None):
+        arr = (ctypes.c_int64 * len(shape))(*shape)
+        key = required_meta_key.encode() if required_meta_key is not None else None
+        _check(lib().veda_selector_check(self._h, n_tensors, arr, len(shape), max_file_bytes, key),
+               "veda_selector_check")
+
+    def check_published(self, hotkey_key: Optional[str] = None) -> None:
+        """The competition layout (hotkey_key: the metadata key that must name the hotkey)."""
+        self.check(PUBLISHED_LAYOUT["n_tensors"], PUBLISHED_LAYOUT["shape"], PUBLISHED_LAYOUT["max_file_bytes"],
+                   hotkey_key)
+
+    def __len__(self) -> int:
+        return lib().veda_selector_count(self._h)
+
+    def info(self, i: int):
+        name, dt, nd = ctypes.c_char_p(), ctypes.c_char_p(), ctypes.c_int32()
+        shape = (ctypes.c_int64 * 8)()
+        _check(lib().veda_selector_info(self._h, i, ctypes.byref(name), ctypes.byref(dt), ctypes.byref(nd), shape),
+               "veda_selector_info")
+        return name.value.decode(), dt.value.decode(), tuple(shape[k] for k in range(nd.value))
+
+    def names(self):
+        return [self.info(i)[0] for i in range(len(self))]
+
+    def metadata(self, key: str) -> Optional[str]:
+        v = lib().veda_selector_metadata(self._h, key.encode())
+        return None if v is None else v.decode()
+
+    def read(self, name: str, dtype=torch.bfloat16, scale: float = 1.0) -> torch.Tensor:
+        idx = ctypes.c_int32()
+        _check(lib().veda_selector_find(self._h, name.encode(), ctypes.byref(idx)), "veda_selector_find")
+        _, _, shape = self.info(idx.value)
+        if dtype not in (torch.float32, torch.bfloat16):
+            raise ValueError("dtype must be float32 or bfloat16")
+        out = torch.empty(shape, dtype=dtype)
+        _check(lib().veda_selector_read(self._h, idx.value, VEDA_F32 if dtype == torch.float32 else VEDA_BF16,
+                                        float(scale), out.data_ptr(), out.numel() * out.element_size()),
+               "veda_selector_read")
+        return out

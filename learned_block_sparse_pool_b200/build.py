@@ -1,4 +1,4 @@
-"""Build libveda.so (all CUDA sources, sm_100a) in the package directory.
+"""Build libveda.so (all CUDA sources, sm_100a, and the host-only C++ sources) in the package directory.
 
     python -m learned_block_sparse_pool_b200.build [--force] [--verbose]
 
@@ -29,7 +29,7 @@ FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", 
 
 
 def sources():
-    return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cpp")))
 
 
 def _headers():

@@ -402,6 +402,8 @@ const char* veda_status_string(veda_status s)
     case VEDA_ERR_CUDA: return "VEDA_ERR_CUDA";
     case VEDA_ERR_TIMEOUT: return "VEDA_ERR_TIMEOUT";
     case VEDA_ERR_BAD_INDEX: return "VEDA_ERR_BAD_INDEX";
+    case VEDA_ERR_FORMAT: return "VEDA_ERR_FORMAT";
+    case VEDA_ERR_IO: return "VEDA_ERR_IO";
     }
     return "VEDA_ERR_UNKNOWN";
 }

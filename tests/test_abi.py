@@ -223,5 +223,6 @@ def test_workspace_view_bounds(L):
 def test_status_strings(L):
     for code, name in [(0, "VEDA_OK"), (-1, "VEDA_ERR_INVALID_ARG"), (-2, "VEDA_ERR_UNSUPPORTED"),
                        (-3, "VEDA_ERR_WORKSPACE"), (-4, "VEDA_ERR_CUDA"), (-5, "VEDA_ERR_TIMEOUT"),
-                       (-6, "VEDA_ERR_BAD_INDEX"), (-99, "VEDA_ERR_UNKNOWN")]:
+                       (-6, "VEDA_ERR_BAD_INDEX"), (-7, "VEDA_ERR_FORMAT"), (-8, "VEDA_ERR_IO"),
+                       (-99, "VEDA_ERR_UNKNOWN")]:
         assert B.status_string(code) == name
