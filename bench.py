@@ -409,25 +409,21 @@ def dense_query_run(args, veda, w, g, p, ws, dev, local, rank, n, dist):
         dist.destroy_process_group()
 
 
-def e2e_run(veda, w, g, p, dev, stream, steps, n, dist, simt):
-    """Same metric through the public fused call (veda_attn) with host
-    buffers: every step copies its inputs from pinned host memory and reads
-    the attention output back."""
-    host = {k: v.cpu().pin_memory() for k, v in g.items()}
-    d = {k: torch.empty_like(v) for k, v in g.items()}
-    p2 = make_problem(veda, w, d, simt)
-    ws = veda.workspace(p2)
-    iv, ir = veda.alloc_indices(p2)
-    out, _ = veda.alloc_output(p2)
-    out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+def e2e_run(veda, w, g, p, dev, stream, steps, n, dist, simt, heads_per_group=2):
+    """Same metric through the public host-buffer call (veda_attn_host): every
+    step takes Q, K, V, the dense and reference keys and the selector weights
+    from pinned host memory and returns the attention output to pinned host
+    memory; the library pipelines the copies with the compute over groups of
+    heads."""
+    host = {k: v.cpu().contiguous().pin_memory() for k, v in g.items()}
+    ph = make_problem(veda, w, host, simt)
+    buf = veda.attn_host_buffer(ph, heads_per_group, dev)
+    out_host = torch.empty((w.B, w.n_video, w.H, w.d), dtype=w.torch_dtype, pin_memory=True)
     h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = out.numel() * out.element_size()
+    d2h = out_host.numel() * out_host.element_size()
 
     def one():
-        for k in host:
-            d[k].copy_(host[k], non_blocking=True)
-        veda.attn(p2, d["w_q"], d["w_k"], iv, ir, out, None, ws, stream)
-        out_host.copy_(out, non_blocking=True)
+        veda.attn_host(ph, host["w_q"], host["w_k"], None, None, out_host, None, heads_per_group, buf, stream)
 
     one()
     torch.cuda.synchronize(dev)
@@ -442,11 +438,11 @@ def e2e_run(veda, w, g, p, dev, stream, steps, n, dist, simt):
     t1.record(stream)
     torch.cuda.synchronize(dev)
     ms = max_over_ranks(dist, [t0.elapsed_time(t1)], dev)[0]
-    st = veda.check_status(ws, stream)
+    st = veda.check_status(buf, stream)
     if st != 0:
         raise RuntimeError(f"device status after e2e: {veda.status_string(st)}")
     return {"value": round(ms / k2 / n, 4), "unit": "ms", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "steps": k2, "call": "veda_attn (fused) with pinned host buffers"}
+            "steps": k2, "call": f"veda_attn_host (pinned host buffers, {heads_per_group} heads per group)"}
 
 
 def run_reference(args, w, dev, n):

@@ -169,6 +169,32 @@ VEDA_API veda_status veda_dense_query_attn(const veda_problem* p, const void* q_
                                   int64_t q_stride_b, int64_t q_stride_tok, int64_t q_stride_h,
                                   void* out, float* lse, void* ws, size_t ws_bytes, veda_stream_t stream);
 
+/* Steps 1-4 on HOST buffers, with the host<->device copies pipelined.
+ * The heads are processed in groups of heads_per_group: while one group's
+ * selection and attention run, the next group's Q/K/V and weights are
+ * copied in and the previous group's output, LSE and kept tiles are copied
+ * out, on three streams forked from and joined back to `stream` (each head
+ * is independent of the others, so a group is a complete problem of its
+ * own).  Results equal veda_attn's.
+ *   p              the problem with HOST pointers; Q and every segment packed
+ *                  [B, n, H, d] (stride_h = d, stride_tok = H d, stride_b =
+ *                  n H d); page-locked host memory lets the copies overlap
+ *   w_q, w_k       HOST [H, d, r]
+ *   idx_video/ref  HOST [B, H, n_q_tiles, budget] int32 out, or idx_video
+ *                  NULL to skip them (idx_ref NULL iff no reference)
+ *   out, lse       HOST [B, video.n_tokens, H, d] / [B, H, video.n_tokens]
+ *                  fp32 (lse may be NULL)
+ *   dev_buf        caller-owned DEVICE buffer of veda_attn_host_buffer_size
+ *                  bytes, 256-byte aligned; its first 256 bytes are a status
+ *                  block: initialise it with veda_workspace_init and read
+ *                  device-side errors with veda_check_status(dev_buf).
+ * Returns after enqueueing.  VEDA_ERR_UNSUPPORTED for host tensors that are
+ * not packed; VEDA_ERR_WORKSPACE for a short or misaligned dev_buf. */
+VEDA_API veda_status veda_attn_host_buffer_size(const veda_problem* p, int32_t heads_per_group, size_t* bytes);
+VEDA_API veda_status veda_attn_host(const veda_problem* p, const void* w_q, const void* w_k, int32_t* idx_video,
+                           int32_t* idx_ref, void* out, float* lse, int32_t heads_per_group, void* dev_buf,
+                           size_t dev_bytes, veda_stream_t stream);
+
 /* Steps 1-4 in one call (selection, then attention on the selected tiles),
  * stream-ordered, no host synchronisation.  idx_video / idx_ref receive the
  * kept tiles as in veda_select_tiles. */

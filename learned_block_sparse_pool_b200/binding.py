@@ -33,7 +33,8 @@ EXPORTS = ("veda_workspace_size", "veda_workspace_init", "veda_select_tiles", "v
            "veda_attn", "veda_pool_project", "veda_score_tiles", "veda_topk_tiles", "veda_workspace_view",
            "veda_check_status", "veda_status_string", "veda_select_tiles_noalloc", "veda_dense_query_attn",
            "veda_selector_open", "veda_selector_close", "veda_selector_check", "veda_selector_count",
-           "veda_selector_find", "veda_selector_info", "veda_selector_metadata", "veda_selector_read")
+           "veda_selector_find", "veda_selector_info", "veda_selector_metadata", "veda_selector_read",
+           "veda_attn_host_buffer_size", "veda_attn_host")
 
 
 class VedaError(RuntimeError):
@@ -85,6 +86,8 @@ def lib() -> ctypes.CDLL:
         L.veda_select_tiles_noalloc.argtypes = [P, vp, vp, i32p, i32p, vp]
         L.veda_status_string.argtypes = [ctypes.c_int]
         L.veda_status_string.restype = ctypes.c_char_p
+        L.veda_attn_host_buffer_size.argtypes = [P, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]
+        L.veda_attn_host.argtypes = [P, vp, vp, i32p, i32p, vp, vp, ctypes.c_int32, vp, sz, vp]
         L.veda_selector_open.argtypes = [ctypes.c_char_p, ctypes.POINTER(vp)]
         L.veda_selector_close.argtypes = [vp]
         L.veda_selector_check.argtypes = [vp, ctypes.c_int32, ctypes.POINTER(ctypes.c_int64), ctypes.c_int32,
@@ -234,6 +237,24 @@ def dense_query_attn(p: Problem, q_rows, out, lse, ws, stream=None) -> None:
     sb, st, sh, _ = q_rows.stride()
     _check(lib().veda_dense_query_attn(p.ref(), q_rows.data_ptr(), n, sb, st, sh, out.data_ptr(), _ptr(lse),
                                        ws.data_ptr(), ws.numel(), _stream(stream)), "veda_dense_query_attn")
+
+
+def attn_host_buffer(p: Problem, heads_per_group: int, device=None) -> torch.Tensor:
+    """The device buffer veda_attn_host needs for problem p (host tensors),
+    with its status block initialised."""
+    n = ctypes.c_size_t()
+    _check(lib().veda_attn_host_buffer_size(p.ref(), heads_per_group, ctypes.byref(n)), "veda_attn_host_buffer_size")
+    buf = torch.empty(n.value, dtype=torch.uint8, device=device or torch.device("cuda"))
+    _check(lib().veda_workspace_init(buf.data_ptr(), buf.numel(), None), "veda_workspace_init")
+    return buf
+
+
+def attn_host(p: Problem, w_q, w_k, idx_v, idx_r, out, lse, heads_per_group: int, dev_buf, stream=None) -> None:
+    """veda_attn on host tensors (p built from host tensors), copies pipelined
+    with the compute over head groups."""
+    _check(lib().veda_attn_host(p.ref(), w_q.data_ptr(), w_k.data_ptr(), _ptr(idx_v), _ptr(idx_r), out.data_ptr(),
+                                _ptr(lse), heads_per_group, dev_buf.data_ptr(), dev_buf.numel(), _stream(stream)),
+           "veda_attn_host")
 
 
 def attn(p: Problem, w_q, w_k, idx_v, idx_r, out, lse, ws, stream=None) -> None:

@@ -178,11 +178,11 @@ veda_status do_score(const veda_problem& p, const Layout& L, void* ws, cudaStrea
 }
 
 veda_status do_topk(const veda_problem& p, const Layout& L, int32_t* idx_v, int32_t* idx_r, void* ws,
-                    cudaStream_t s)
+                    cudaStream_t s, uint32_t* status = nullptr)
 {
     if (!idx_v || (L.nr > 0) != (idx_r != nullptr)) return VEDA_ERR_INVALID_ARG;
     TopkParams T;
-    T.status = at<uint32_t>(ws, 0);
+    T.status = status ? status : at<uint32_t>(ws, 0);
     T.rows = (int64_t)p.B * p.H * L.nq;
     T.scores = at<float>(ws, L.sc_v);
     T.ld = L.ld_v;
@@ -202,7 +202,7 @@ veda_status do_topk(const veda_problem& p, const Layout& L, int32_t* idx_v, int3
 }
 
 veda_status do_attn(const veda_problem& p, const Layout& L, const int32_t* idx_v, const int32_t* idx_r,
-                    void* out, float* lse, void* ws, cudaStream_t s)
+                    void* out, float* lse, void* ws, cudaStream_t s, uint32_t* status = nullptr)
 {
     if (!idx_v || (L.nr > 0) != (idx_r != nullptr)) return VEDA_ERR_INVALID_ARG;
     if (!out || !aligned16(out) || (lse && ((uintptr_t)lse & 3u))) return VEDA_ERR_INVALID_ARG;
@@ -223,7 +223,7 @@ veda_status do_attn(const veda_problem& p, const Layout& L, const int32_t* idx_v
     A.B = p.B; A.H = p.H; A.d = p.d; A.T = p.tile; A.nq = (int32_t)L.nq;
     A.dtype = p.dtype;
     A.scale = p.softmax_scale > 0.f ? p.softmax_scale : 1.0f / sqrtf((float)p.d);
-    A.status = at<uint32_t>(ws, 0);
+    A.status = status ? status : at<uint32_t>(ws, 0);
     A.short_waits = (p.flags & VEDA_FLAG_TEST_SHORT_WAITS) ? 1 : 0;
     if (!(p.flags & VEDA_FLAG_SIMT_ATTENTION) && attn_tc_supported(A)) return from_cuda(launch_attn_tc(A, s));
     return from_cuda(launch_attn_simt(A, s));
@@ -259,6 +259,89 @@ veda_status do_dense_query_attn(const veda_problem& p, const void* q_rows, int64
     A.short_waits = (p.flags & VEDA_FLAG_TEST_SHORT_WAITS) ? 1 : 0;
     if (!(p.flags & VEDA_FLAG_SIMT_ATTENTION) && attn_tc_supported(A)) return from_cuda(launch_attn_tc(A, s));
     return from_cuda(launch_attn_simt(A, s));
+}
+
+
+// ---- host-buffer call: head groups pipelined over three streams ---------
+// The caller's device buffer: a 256-byte status block, then two slots, each
+// holding one head group's inputs, weights, indices, output and workspace.
+struct HostSlot {
+    size_t q, kv[6], wq, wk, iv, ir, out, lse, ws, total;   // offsets inside a slot
+};
+
+// [B, n, H, d] with nothing between rows: the head range of a group is then a
+// 2-D block of B * n rows.
+bool packed(const void* base, int64_t B, int64_t n, int64_t H, int64_t d, int64_t sb, int64_t st, int64_t sh)
+{
+    return base && sh == d && st == H * d && (sb == n * H * d || B == 1);
+}
+
+// The hc-head sub-problem of slot `slot` (device pointers, packed [B, n, hc, d]).
+veda_problem sub_problem(const veda_problem& p, int hc, char* slot, const HostSlot& S)
+{
+    veda_problem c = p;
+    c.H = hc;
+    auto seg = [&](veda_segment& sg, size_t ok, size_t ov) {
+        if (sg.n_tokens == 0) return;
+        sg.k = slot + ok;
+        sg.v = slot + ov;
+        sg.stride_h = p.d;
+        sg.stride_tok = (int64_t)hc * p.d;
+        sg.stride_b = sg.n_tokens * hc * p.d;
+    };
+    c.q = slot + S.q;
+    c.q_stride_h = p.d;
+    c.q_stride_tok = (int64_t)hc * p.d;
+    c.q_stride_b = p.video.n_tokens * hc * p.d;
+    seg(c.video, S.kv[0], S.kv[1]);
+    seg(c.ref, S.kv[2], S.kv[3]);
+    seg(c.dense, S.kv[4], S.kv[5]);
+    return c;
+}
+
+HostSlot host_slot(const veda_problem& p, int hc)
+{
+    HostSlot S;
+    const size_t es = esize(p.dtype);
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at_ = off;
+        off = align_up(off + bytes, kAlign);
+        return at_;
+    };
+    const size_t row = (size_t)hc * p.d * es;
+    S.q = take((size_t)p.B * p.video.n_tokens * row);
+    const veda_segment* segs[3] = {&p.video, &p.ref, &p.dense};
+    for (int g = 0; g < 3; ++g) {
+        S.kv[2 * g] = take((size_t)p.B * segs[g]->n_tokens * row);
+        S.kv[2 * g + 1] = take((size_t)p.B * segs[g]->n_tokens * row);
+    }
+    S.wq = take((size_t)hc * p.d * p.r * es);
+    S.wk = take((size_t)hc * p.d * p.r * es);
+    veda_problem c = p;
+    c.H = hc;
+    const Layout L = layout(c);
+    S.iv = take(sizeof(int32_t) * (size_t)p.B * hc * L.nq * p.video.budget);
+    S.ir = take(sizeof(int32_t) * (size_t)p.B * hc * L.nq * (L.nr > 0 ? p.ref.budget : 0));
+    S.out = take((size_t)p.B * p.video.n_tokens * row);
+    S.lse = take(sizeof(float) * (size_t)p.B * hc * p.video.n_tokens);
+    S.ws = take(L.total);
+    S.total = off;
+    return S;
+}
+
+veda_status check_host_problem(const veda_problem& p, int heads_per_group)
+{
+    if (heads_per_group < 1) return VEDA_ERR_INVALID_ARG;
+    if (!packed(p.q, p.B, p.video.n_tokens, p.H, p.d, p.q_stride_b, p.q_stride_tok, p.q_stride_h))
+        return VEDA_ERR_UNSUPPORTED;
+    const veda_segment* segs[3] = {&p.video, &p.ref, &p.dense};
+    for (auto* sg : segs)
+        if (sg->n_tokens > 0 &&
+            (!packed(sg->k, p.B, sg->n_tokens, p.H, p.d, sg->stride_b, sg->stride_tok, sg->stride_h) ||
+             !packed(sg->v, p.B, sg->n_tokens, p.H, p.d, sg->stride_b, sg->stride_tok, sg->stride_h)))
+            return VEDA_ERR_UNSUPPORTED;
+    return VEDA_OK;
 }
 
 }  // namespace
@@ -345,6 +428,140 @@ veda_status veda_dense_query_attn(const veda_problem* p, const void* q_rows, int
     if (!ws || ((uintptr_t)ws % kAlign) != 0 || ws_bytes < kAlign) return VEDA_ERR_WORKSPACE;
     return do_dense_query_attn(*p, q_rows, n_rows, q_stride_b, q_stride_tok, q_stride_h, out, lse, ws,
                                (cudaStream_t)stream);
+}
+
+veda_status veda_attn_host_buffer_size(const veda_problem* p, int32_t heads_per_group, size_t* bytes)
+{
+    if (!bytes) return VEDA_ERR_INVALID_ARG;
+    veda_status st = validate(p);
+    if (st != VEDA_OK) return st;
+    if ((st = check_host_problem(*p, heads_per_group)) != VEDA_OK) return st;
+    const int hc = heads_per_group < p->H ? heads_per_group : p->H;
+    *bytes = kAlign + 2 * host_slot(*p, hc).total;
+    return VEDA_OK;
+}
+
+veda_status veda_attn_host(const veda_problem* p, const void* w_q, const void* w_k, int32_t* idx_video,
+                           int32_t* idx_ref, void* out, float* lse, int32_t heads_per_group, void* dev_buf,
+                           size_t dev_bytes, veda_stream_t stream)
+{
+    veda_status st = validate(p);
+    if (st != VEDA_OK) return st;
+    if ((st = check_host_problem(*p, heads_per_group)) != VEDA_OK) return st;
+    const veda_problem& P = *p;
+    const int hc = heads_per_group < P.H ? heads_per_group : P.H;
+    const HostSlot S = host_slot(P, hc);
+    if (!dev_buf || ((uintptr_t)dev_buf % kAlign) != 0 || dev_bytes < kAlign + 2 * S.total) return VEDA_ERR_WORKSPACE;
+    if (!w_q || !w_k || !out || (lse && ((uintptr_t)lse & 3u))) return VEDA_ERR_INVALID_ARG;
+    if ((P.ref.n_tokens > 0) != (idx_ref != nullptr) && idx_video) return VEDA_ERR_INVALID_ARG;
+    const size_t es = esize(P.dtype);
+    const int64_t nq = (P.video.n_tokens + P.tile - 1) / P.tile;
+    uint32_t* status = static_cast<uint32_t*>(dev_buf);
+    char* slots[2] = {static_cast<char*>(dev_buf) + kAlign, static_cast<char*>(dev_buf) + kAlign + S.total};
+    cudaStream_t caller = (cudaStream_t)stream;
+
+    // three streams (copy in, compute, copy out) forked from and joined back to the caller's stream
+    cudaStream_t sin = nullptr, scomp = nullptr, sout = nullptr;
+    cudaEvent_t ev[9] = {};
+    bool ok = cudaStreamCreateWithFlags(&sin, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&scomp, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&sout, cudaStreamNonBlocking) == cudaSuccess;
+    for (int i = 0; i < 9 && ok; ++i) ok = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) == cudaSuccess;
+    cudaEvent_t &e_fork = ev[0], &e_in0 = ev[1], &e_in1 = ev[2], &e_c0 = ev[3], &e_c1 = ev[4], &e_free0 = ev[5],
+                &e_free1 = ev[6], &e_comp_end = ev[7], &e_out_end = ev[8];
+    cudaEvent_t e_in[2] = {e_in0, e_in1}, e_comp[2] = {e_c0, e_c1}, e_free[2] = {e_free0, e_free1};
+    st = ok ? VEDA_OK : VEDA_ERR_CUDA;
+    if (st == VEDA_OK) {
+        ok = cudaEventRecord(e_fork, caller) == cudaSuccess && cudaStreamWaitEvent(sin, e_fork, 0) == cudaSuccess &&
+             cudaStreamWaitEvent(scomp, e_fork, 0) == cudaSuccess &&
+             cudaStreamWaitEvent(sout, e_fork, 0) == cudaSuccess;
+        if (!ok) st = VEDA_ERR_CUDA;
+    }
+    const veda_segment* hsegs[3] = {&P.video, &P.ref, &P.dense};
+    for (int h0 = 0, c = 0; h0 < P.H && st == VEDA_OK; h0 += hc, ++c) {
+        const int g = P.H - h0 < hc ? P.H - h0 : hc;   // heads in this group
+        const int sl = c & 1;
+        char* slot = slots[sl];
+        bool k_ok = true;
+        // ---- copy in (after the slot's previous group has been copied out) ----
+        if (c >= 2) k_ok = cudaStreamWaitEvent(sin, e_free[sl], 0) == cudaSuccess;
+        const size_t row = (size_t)g * P.d * es, hrow = (size_t)P.H * P.d * es, drow = (size_t)hc * P.d * es;
+        auto in2d = [&](size_t off, const void* host, int64_t n) {
+            if (n > 0 && k_ok)
+                k_ok = cudaMemcpy2DAsync(slot + off, drow, static_cast<const char*>(host) + (size_t)h0 * P.d * es,
+                                         hrow, row, (size_t)P.B * n, cudaMemcpyHostToDevice, sin) == cudaSuccess;
+        };
+        in2d(S.q, P.q, P.video.n_tokens);
+        for (int s3 = 0; s3 < 3; ++s3) {
+            in2d(S.kv[2 * s3], hsegs[s3]->k, hsegs[s3]->n_tokens);
+            in2d(S.kv[2 * s3 + 1], hsegs[s3]->v, hsegs[s3]->n_tokens);
+        }
+        const size_t wbytes = (size_t)g * P.d * P.r * es;
+        if (k_ok) k_ok = cudaMemcpyAsync(slot + S.wq, static_cast<const char*>(w_q) + (size_t)h0 * P.d * P.r * es,
+                                         wbytes, cudaMemcpyHostToDevice, sin) == cudaSuccess;
+        if (k_ok) k_ok = cudaMemcpyAsync(slot + S.wk, static_cast<const char*>(w_k) + (size_t)h0 * P.d * P.r * es,
+                                         wbytes, cudaMemcpyHostToDevice, sin) == cudaSuccess;
+        if (k_ok) k_ok = cudaEventRecord(e_in[sl], sin) == cudaSuccess;
+        // ---- compute the group's selection and attention ----
+        veda_problem cp = sub_problem(P, hc, slot, S);
+        cp.H = g;
+        // the group's tensors are packed for hc heads; a short last group keeps that layout
+        cp.q_stride_tok = (int64_t)hc * P.d;
+        const Layout L = layout(cp);
+        void* ws = slot + S.ws;
+        int32_t* iv = reinterpret_cast<int32_t*>(slot + S.iv);
+        int32_t* ir = L.nr > 0 ? reinterpret_cast<int32_t*>(slot + S.ir) : nullptr;
+        if (k_ok) k_ok = cudaStreamWaitEvent(scomp, e_in[sl], 0) == cudaSuccess;
+        if (!k_ok) { st = VEDA_ERR_CUDA; break; }
+        if ((st = do_pool_project(cp, L, slot + S.wq, slot + S.wk, ws, scomp)) != VEDA_OK) break;
+        if ((st = do_score(cp, L, ws, scomp)) != VEDA_OK) break;
+        if ((st = do_topk(cp, L, iv, ir, ws, scomp, status)) != VEDA_OK) break;
+        if ((st = do_attn(cp, L, iv, ir, slot + S.out, lse ? reinterpret_cast<float*>(slot + S.lse) : nullptr, ws,
+                          scomp, status)) != VEDA_OK)
+            break;
+        k_ok = cudaEventRecord(e_comp[sl], scomp) == cudaSuccess &&
+               cudaStreamWaitEvent(sout, e_comp[sl], 0) == cudaSuccess;
+        // ---- copy out: output rows, LSE rows and kept tiles of the group's heads ----
+        // the group's output is packed for its own g heads
+        if (k_ok) k_ok = cudaMemcpy2DAsync(static_cast<char*>(out) + (size_t)h0 * P.d * es, hrow, slot + S.out, row,
+                                           row, (size_t)P.B * P.video.n_tokens, cudaMemcpyDeviceToHost,
+                                           sout) == cudaSuccess;
+        if (k_ok && lse) {
+            const size_t w4 = sizeof(float) * (size_t)g * P.video.n_tokens;
+            k_ok = cudaMemcpy2DAsync(lse + (size_t)h0 * P.video.n_tokens, sizeof(float) * (size_t)P.H * P.video.n_tokens,
+                                     slot + S.lse, sizeof(float) * (size_t)g * P.video.n_tokens, w4, (size_t)P.B,
+                                     cudaMemcpyDeviceToHost, sout) == cudaSuccess;
+        }
+        if (k_ok && idx_video) {
+            const size_t wv = sizeof(int32_t) * (size_t)g * nq * P.video.budget;
+            k_ok = cudaMemcpy2DAsync(idx_video + (size_t)h0 * nq * P.video.budget,
+                                     sizeof(int32_t) * (size_t)P.H * nq * P.video.budget, iv, wv, wv, (size_t)P.B,
+                                     cudaMemcpyDeviceToHost, sout) == cudaSuccess;
+            if (k_ok && ir) {
+                const size_t wr = sizeof(int32_t) * (size_t)g * nq * P.ref.budget;
+                k_ok = cudaMemcpy2DAsync(idx_ref + (size_t)h0 * nq * P.ref.budget,
+                                         sizeof(int32_t) * (size_t)P.H * nq * P.ref.budget, ir, wr, wr, (size_t)P.B,
+                                         cudaMemcpyDeviceToHost, sout) == cudaSuccess;
+            }
+        }
+        if (k_ok) k_ok = cudaEventRecord(e_free[sl], sout) == cudaSuccess;
+        if (!k_ok) st = VEDA_ERR_CUDA;
+    }
+    // join: the caller's stream waits for every copy and kernel of this call
+    if (sin && scomp && sout && ev[7] && ev[8]) {
+        cudaEventRecord(e_comp_end, scomp);
+        cudaEventRecord(e_out_end, sout);
+        cudaStreamWaitEvent(caller, e_comp_end, 0);
+        cudaStreamWaitEvent(caller, e_out_end, 0);
+        cudaEventRecord(e_fork, sin);               // the copy-in stream's last work
+        cudaStreamWaitEvent(caller, e_fork, 0);
+    }
+    for (int i = 0; i < 9; ++i)
+        if (ev[i]) cudaEventDestroy(ev[i]);         // released once their work completes
+    if (sin) cudaStreamDestroy(sin);
+    if (scomp) cudaStreamDestroy(scomp);
+    if (sout) cudaStreamDestroy(sout);
+    return st;
 }
 
 veda_status veda_attn(const veda_problem* p, const void* w_q, const void* w_k, int32_t* idx_video,
