@@ -208,6 +208,29 @@ def test_dense_query_arguments_checked(L):
     assert L.veda_dense_query_attn(ctypes.byref(q_bad), *ok) == B.VEDA_ERR_UNSUPPORTED
 
 
+def test_host_call_buffer_and_arguments(L):
+    """veda_attn_host: buffer size and the checks made before any CUDA call."""
+    p = _problem()                      # packed [B, N, H, d] host layout, reference + dense present
+    n1, n4 = B.ctypes.c_size_t(), B.ctypes.c_size_t()
+    assert L.veda_attn_host_buffer_size(B.ctypes.byref(p), 1, B.ctypes.byref(n1)) == B.VEDA_OK
+    assert L.veda_attn_host_buffer_size(B.ctypes.byref(p), 4, B.ctypes.byref(n4)) == B.VEDA_OK
+    assert 256 < n1.value < n4.value    # status block + two slots; a slot grows with the group
+    assert L.veda_attn_host_buffer_size(B.ctypes.byref(p), 9, B.ctypes.byref(n1)) == B.VEDA_OK
+    assert n1.value == n4.value         # groups are capped at H heads
+    assert L.veda_attn_host_buffer_size(B.ctypes.byref(p), 0, B.ctypes.byref(n1)) == B.VEDA_ERR_INVALID_ARG
+    unpacked = _problem(q_stride_tok=4 * 128 * 2)
+    assert L.veda_attn_host_buffer_size(B.ctypes.byref(unpacked), 2, B.ctypes.byref(n1)) == B.VEDA_ERR_UNSUPPORTED
+    buf, w, idx, out = 0x10000000, 0x900000, 0x500000, 0xA00000
+
+    def call(prob, *, dev_bytes=n4.value, dev=buf, o=out, wq=w):
+        return L.veda_attn_host(B.ctypes.byref(prob), wq, w, None, None, o, None, 4, dev, dev_bytes, None)
+    assert call(p, dev_bytes=n4.value - 1) == B.VEDA_ERR_WORKSPACE
+    assert call(p, dev=buf + 16) == B.VEDA_ERR_WORKSPACE
+    assert call(p, o=0) == B.VEDA_ERR_INVALID_ARG
+    assert call(p, wq=0) == B.VEDA_ERR_INVALID_ARG
+    assert call(unpacked) == B.VEDA_ERR_UNSUPPORTED
+
+
 def test_workspace_view_bounds(L):
     p = _problem(**{"ref.n_tokens": 0, "ref.budget": 0})
     st, n = _ws_size(L, p)
