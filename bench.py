@@ -195,6 +195,9 @@ def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
+    if args.gpus != world:
+        raise SystemExit(f"--gpus {args.gpus} needs one process per GPU: launch with "
+                         f"torch.distributed.run --nproc-per-node {args.gpus} (WORLD_SIZE is {world})")
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         # the CPU oracle: rank 0 alone runs and prints; other ranks do no work
