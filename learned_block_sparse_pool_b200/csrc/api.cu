@@ -229,9 +229,27 @@ veda_status do_attn(const veda_problem& p, const Layout& L, const int32_t* idx_v
     return from_cuda(launch_attn_simt(A, s));
 }
 
+// Key-range split for few (b, h, query tile) units: the number of ranges S
+// (1..4) that minimises the waves of the persistent grid per unit of work,
+// with a 5% charge for the merge.
+int choose_split(int64_t units, int n_list)
+{
+    const int64_t sms = num_sms();
+    int best = 1;
+    double best_cost = (double)((units + sms - 1) / sms);
+    for (int S = 2; S <= 4 && 2 * S <= n_list; ++S) {
+        const double cost = (double)((units * S + sms - 1) / sms) / S * 1.05;
+        if (cost < best_cost) {
+            best = S;
+            best_cost = cost;
+        }
+    }
+    return best;
+}
+
 // Dense-query rows: every query row attends to every token of every segment.
 veda_status do_dense_query_attn(const veda_problem& p, const void* q_rows, int64_t n_rows, int64_t sb, int64_t st,
-                                int64_t sh, void* out, float* lse, void* ws, cudaStream_t s)
+                                int64_t sh, void* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t s)
 {
     const size_t es = esize(p.dtype);
     if (n_rows < 1 || n_rows > (int64_t)1 << 30 || !q_rows || !aligned16(q_rows)) return VEDA_ERR_INVALID_ARG;
@@ -257,7 +275,20 @@ veda_status do_dense_query_attn(const veda_problem& p, const void* q_rows, int64
     A.scale = p.softmax_scale > 0.f ? p.softmax_scale : 1.0f / sqrtf((float)p.d);
     A.status = at<uint32_t>(ws, 0);
     A.short_waits = (p.flags & VEDA_FLAG_TEST_SHORT_WAITS) ? 1 : 0;
-    if (!(p.flags & VEDA_FLAG_SIMT_ATTENTION) && attn_tc_supported(A)) return from_cuda(launch_attn_tc(A, s));
+    if (!(p.flags & VEDA_FLAG_SIMT_ATTENTION) && attn_tc_supported(A)) {
+        // few units: split every key list over S CTAs and merge, with the
+        // partial results in the workspace past its status block (if they fit)
+        const int S = choose_split((int64_t)A.B * A.H * A.nq, A.k_v + A.k_r + A.dense.n_tiles);
+        const size_t rows = (size_t)A.B * A.H * (size_t)n_rows;
+        const size_t o_bytes = align_up(sizeof(float) * S * rows * p.d, kAlign);
+        const size_t ml_bytes = align_up(sizeof(float) * 2 * S * rows, kAlign);
+        if (S > 1 && kAlign + o_bytes + ml_bytes <= ws_bytes) {
+            A.n_split = S;
+            A.part_o = at<float>(ws, kAlign);
+            A.part_ml = at<float>(ws, kAlign + o_bytes);
+        }
+        return from_cuda(launch_attn_tc(A, s));
+    }
     return from_cuda(launch_attn_simt(A, s));
 }
 
@@ -426,7 +457,7 @@ veda_status veda_dense_query_attn(const veda_problem* p, const void* q_rows, int
     veda_status st = validate(p);
     if (st != VEDA_OK) return st;
     if (!ws || ((uintptr_t)ws % kAlign) != 0 || ws_bytes < kAlign) return VEDA_ERR_WORKSPACE;
-    return do_dense_query_attn(*p, q_rows, n_rows, q_stride_b, q_stride_tok, q_stride_h, out, lse, ws,
+    return do_dense_query_attn(*p, q_rows, n_rows, q_stride_b, q_stride_tok, q_stride_h, out, lse, ws, ws_bytes,
                                (cudaStream_t)stream);
 }
 

@@ -74,7 +74,32 @@ struct TcParams {
     float scale_log2;
     uint32_t* status;
     long long wait_limit;       // clocks a pipeline wait may take before the CTA aborts
+    int32_t n_split;            // >1: each (b, h, query tile) is split into n_split key ranges
+    float* part_o;              // [n_split][B H][n_qtok][D] unnormalised O of each range
+    float* part_ml;             // [n_split][B H][n_qtok][2] (max in base-2 units, sum) of each range
 };
+
+// A work unit: (b, h, query tile i) and, when the kept list is split, the
+// range [j0, j0 + nl) of it that this unit covers.
+struct UnitRef {
+    int64_t row;                // (b H + h) nq + i: the kept-list row
+    int i, h, b, s, j0, nl;
+};
+
+template <bool kSplit>
+__device__ __forceinline__ UnitRef unit_ref(const TcParams& P, int64_t u, int n_list)
+{
+    UnitRef r;
+    r.row = kSplit ? u / P.n_split : u;
+    r.s = kSplit ? (int)(u % P.n_split) : 0;
+    r.i = (int)(r.row % P.nq);
+    const int64_t bh = r.row / P.nq;
+    r.h = (int)(bh % P.H);
+    r.b = (int)(bh / P.H);
+    r.j0 = kSplit ? (int)((int64_t)r.s * n_list / P.n_split) : 0;
+    r.nl = kSplit ? (int)((int64_t)(r.s + 1) * n_list / P.n_split) - r.j0 : n_list;
+    return r;
+}
 
 struct __align__(1024) Smem {
     uint8_t q[kTileBytes];
@@ -351,6 +376,7 @@ __device__ __forceinline__ void load_box_pair(const TcParams& P, int m, uint8_t*
 }
 
 // --------------------------------------------------------------- kernel ---
+template <bool kSplit>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ TcParams P)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -395,16 +421,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         uint32_t uq = 0, f = 0;
         bool ok = true;
         for (int64_t u = blockIdx.x; u < P.units && ok; u += gridDim.x) {
-            const int i = (int)(u % P.nq);
-            const int64_t bh = u / P.nq;
-            const int h = (int)(bh % P.H), b = (int)(bh / P.H);
+            const UnitRef ur = unit_ref<kSplit>(P, u, n_list);
+            const int i = ur.i, h = ur.h, b = ur.b;
+            const int nl = kSplit ? ur.nl : n_list, j0 = kSplit ? ur.j0 : 0;
+            const int64_t urow = kSplit ? ur.row : u;
             // the previous unit's last S has read the Q buffer
             if (uq >= 1 && !(ok = wait_phase(sm, &sm.q_empty, (uq - 1) & 1, P.status, P.wait_limit))) break;
             mbar_expect_tx(&sm.q_full, kTileBytes);
             load_box_pair(P, 0, sm.q, &sm.q_full, h, i * TT, b);
             ++uq;
             auto load_kv = [&](int j, int which) -> bool {
-                const TileRef r = resolve(P, u, j);
+                const TileRef r = resolve(P, urow, j0 + j);
                 const uint32_t st = f % NS;
                 if (f >= NS && !wait_phase(sm, &sm.kv_empty[st], ((f / NS) - 1) & 1, P.status, P.wait_limit)) return false;
                 mbar_expect_tx(&sm.kv_full[st], kTileBytes);
@@ -415,8 +442,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             };
             // the MMA warp's consumption order: K0, K1, V0, K2, V1, ..., V(n-1)
             if (!(ok = load_kv(0, 0))) break;
-            for (int j = 0; j < n_list && ok; ++j) {
-                if (j + 1 < n_list) ok = load_kv(j + 1, 0);
+            for (int j = 0; j < nl && ok; ++j) {
+                if (j + 1 < nl) ok = load_kv(j + 1, 0);
                 if (ok) ok = load_kv(j, 1);
             }
         }
@@ -439,6 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         };
         bool ok = true;
         for (int64_t u = blockIdx.x; u < P.units && ok; u += gridDim.x) {
+            const int nl = kSplit ? unit_ref<kSplit>(P, u, n_list).nl : n_list;
             if (!(ok = warp_wait(sm, &sm.q_full, uq & 1, P.status, P.wait_limit))) break;
             ++uq;
             tc_fence_after();
@@ -456,13 +484,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 }
                 umma_commit(&sm.s_full[g]);
                 umma_commit(&sm.kv_empty[st]);
-                if (j == n_list - 1) umma_commit(&sm.q_empty);   // last read of this Q tile
+                if (j == nl - 1) umma_commit(&sm.q_empty);   // last read of this Q tile
                 ring_next();
                 return true;
             };
             if (!(ok = issue_s(0))) break;
-            if (n_list > 1 && !(ok = issue_s(1))) break;
-            for (int j = 0; j < n_list && ok; ++j) {
+            if (nl > 1 && !(ok = issue_s(1))) break;
+            for (int j = 0; j < nl && ok; ++j) {
                 const uint32_t g = j & 1, st = kst;
                 if (!(ok = warp_wait(sm, &sm.kv_full[st], kph, P.status, P.wait_limit))) break;
                 if (!(ok = warp_wait(sm, &sm.p_full[g], (g ? pc1 : pc0) & 1, P.status, P.wait_limit))) break;
@@ -479,7 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 umma_commit(&sm.kv_empty[st]);
                 ring_next();
                 if (g) ++pc1; else ++pc0;
-                if (j + 2 < n_list && !(ok = issue_s(j + 2))) break;
+                if (j + 2 < nl && !(ok = issue_s(j + 2))) break;
             }
             ++units_done;
         }
@@ -499,15 +527,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         uint32_t sc = 0, uu = 0;          // S tiles consumed by this group; units done
         bool ok = true;
         for (int64_t u = blockIdx.x; u < P.units && ok; u += gridDim.x, ++uu) {
-            const int i = (int)(u % P.nq);
-            const int64_t bh = u / P.nq;
-            const int h = (int)(bh % P.H), b = (int)(bh / P.H);
+            const UnitRef ur = unit_ref<kSplit>(P, u, n_list);
+            const int i = ur.i, h = ur.h, b = ur.b;
+            const int nl = kSplit ? ur.nl : n_list, j0 = kSplit ? ur.j0 : 0;
+            const int64_t urow = kSplit ? ur.row : u;
             float m_run = -INFINITY, l = 0.f;
             int cnt = 0;
-            TileRef r_next = resolve(P, u, g);
-            for (int j = g; j < n_list; j += 2, ++sc, ++cnt) {
+            TileRef r_next = resolve(P, urow, j0 + g);
+            for (int j = g; j < nl; j += 2, ++sc, ++cnt) {
                 const TileRef r = r_next;
-                if (j + 2 < n_list) r_next = resolve(P, u, j + 2);   // one tile ahead
+                if (j + 2 < nl) r_next = resolve(P, urow, j0 + j + 2);   // one tile ahead
                 if (!(ok = warp_wait(sm, &sm.s_full[g], sc & 1, P.status, P.wait_limit))) break;
                 tc_fence_after();
                 uint32_t s[128];
@@ -613,9 +642,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             const float f0 = (m0 == -INFINITY) ? 0.f : fast_exp2(m0 - M);
             const float f1 = (m1 == -INFINITY) ? 0.f : fast_exp2(m1 - M);
             const float L = l0 * f0 + l1 * f1;
-            const float inv = 1.f / L;
+            constexpr bool split = kSplit;
+            const float inv = split ? 1.f : 1.f / L;   // a split range stays unnormalised for the merge
             const float c0 = f0 * inv, c1 = f1 * inv;
             const int64_t tok = (int64_t)i * TT + row;
+            const int64_t prow = kSplit ? (((u % P.n_split) * P.B + b) * (int64_t)P.H + h) * P.n_qtok + tok : 0;
             __nv_bfloat16* dst = P.out + (((int64_t)b * P.n_qtok + tok) * P.H + h) * D + 64 * g;
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
@@ -623,7 +654,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 TMEM_LD32(tmem + lane_off + col_o(0) + 64 * g + 32 * q, o0);
                 TMEM_LD32(tmem + lane_off + col_o(1) + 64 * g + 32 * q, o1);
                 tmem_wait_ld();
-                if (tok < P.n_qtok) {
+                if (split && tok < P.n_qtok) {
+                    float* po = P.part_o + prow * D + 64 * g + 32 * q;
+#pragma unroll
+                    for (int c = 0; c < 32; c += 4) {
+                        float v[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float a0 = __uint_as_float(o0[c + e]) * c0;
+                            v[e] = (c1 != 0.f) ? fmaf(__uint_as_float(o1[c + e]), c1, a0) : a0;
+                        }
+                        *reinterpret_cast<float4*>(po + c) = make_float4(v[0], v[1], v[2], v[3]);
+                    }
+                } else if (tok < P.n_qtok) {
 #pragma unroll
                     for (int c = 0; c < 32; c += 8) {
                         float v[8];
@@ -647,8 +690,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                     }
                 }
             }
-            if (P.lse && g == 0 && tok < P.n_qtok)
+            if (split) {
+                if (g == 0 && tok < P.n_qtok) {
+                    P.part_ml[2 * prow] = M;
+                    P.part_ml[2 * prow + 1] = L;
+                }
+            } else if (P.lse && g == 0 && tok < P.n_qtok) {
                 P.lse[((int64_t)b * P.H + h) * P.n_qtok + tok] = (M + __log2f(L)) * 0.69314718055994531f;
+            }
             tc_fence_before();
             mbar_arrive(&sm.o_free);
         }
@@ -661,6 +710,45 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     if (warp == kMmaWarp) {
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512) : "memory");
     }
+}
+
+// Merge of split key ranges: per (b, h, query token) row, with the ranges'
+// (max m_s in base-2 units, sum l_s, unnormalised O_s):
+//   M = max m_s,  L = sum l_s 2^(m_s - M),  O = sum O_s 2^(m_s - M) / L.
+// One warp per row, four channels per lane.
+__global__ void __launch_bounds__(256) merge_splits_kernel(const float* __restrict__ part_o,
+                                                          const float* __restrict__ part_ml, int n_split,
+                                                          int64_t rows, int64_t n_qtok, int H,
+                                                          __nv_bfloat16* __restrict__ out, float* __restrict__ lse)
+{
+    const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (r >= rows) return;
+    const int lane = threadIdx.x & 31;
+    float M = -INFINITY;
+    for (int s = 0; s < n_split; ++s) M = fmaxf(M, part_ml[2 * ((int64_t)s * rows + r)]);
+    float L = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < n_split; ++s) {
+        const int64_t pr = (int64_t)s * rows + r;
+        const float m = part_ml[2 * pr];
+        const float w = m == -INFINITY ? 0.f : exp2f(m - M);
+        L = fmaf(part_ml[2 * pr + 1], w, L);
+        const float4 o = *reinterpret_cast<const float4*>(part_o + pr * D + 4 * lane);
+        acc.x = fmaf(o.x, w, acc.x);
+        acc.y = fmaf(o.y, w, acc.y);
+        acc.z = fmaf(o.z, w, acc.z);
+        acc.w = fmaf(o.w, w, acc.w);
+    }
+    const float inv = 1.f / L;
+    const int64_t bh = r / n_qtok, tok = r % n_qtok;
+    const int64_t b = bh / H, h = bh % H;
+    __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+    uint2 w2;
+    w2.x = *reinterpret_cast<uint32_t*>(&lo);
+    w2.y = *reinterpret_cast<uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(out + ((b * n_qtok + tok) * H + h) * D + 4 * lane) = w2;
+    if (lse && lane == 0) lse[bh * n_qtok + tok] = (M + __log2f(L)) * 0.69314718055994531f;
 }
 
 // ------------------------------------------------------------------ host ---
@@ -725,7 +813,9 @@ bool attn_tc_supported(const AttnParams& p)
 
 cudaError_t launch_attn_tc(const AttnParams& a, cudaStream_t s)
 {
-    const int64_t units = (int64_t)a.B * a.H * a.nq;
+    const int n_split = a.n_split > 1 ? a.n_split : 1;
+    if (n_split > 1 && (!a.part_o || !a.part_ml)) return cudaErrorInvalidValue;
+    const int64_t units = (int64_t)a.B * a.H * a.nq * n_split;
     if (units == 0) return cudaSuccess;
     auto enc = encode_fn();
     if (!enc) return cudaErrorNotSupported;
@@ -766,13 +856,24 @@ cudaError_t launch_attn_tc(const AttnParams& a, cudaStream_t s)
     P.scale_log2 = a.scale * 1.4426950408889634f;
     P.status = a.status;
     P.wait_limit = a.short_waits ? 64 : kWaitLimit;
+    P.n_split = n_split;
+    P.part_o = a.part_o;
+    P.part_ml = a.part_ml;
 
     const size_t smem = sizeof(Smem) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = n_split > 1 ? attn_tc_kernel<true> : attn_tc_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int64_t grid = num_sms();
     if (grid > units) grid = units;
-    attn_tc_kernel<<<(unsigned)grid, kThreads, smem, s>>>(P);
+    kern<<<(unsigned)grid, kThreads, smem, s>>>(P);
+    if (n_split > 1) {
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        const int64_t rows = (int64_t)a.B * a.H * a.n_qtok;
+        merge_splits_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(a.part_o, a.part_ml, n_split, rows, a.n_qtok,
+                                                                       a.H, P.out, a.lse);
+    }
     return cudaGetLastError();
 }
 

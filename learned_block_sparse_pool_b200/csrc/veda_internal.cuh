@@ -86,6 +86,12 @@ struct AttnParams {
     float scale;            // softmax scale (natural-log units)
     uint32_t* status;
     int32_t short_waits;    // test hook: bounded waits give up after ~64 clocks
+    // tensor-core path only: split each (b, h, query tile) key list into n_split
+    // ranges on different CTAs, merged afterwards (scratch: part_o
+    // [n_split][B H][n_qtok][d] fp32, part_ml [n_split][B H][n_qtok][2] fp32)
+    int32_t n_split;
+    float* part_o;
+    float* part_ml;
 };
 
 cudaError_t launch_attn_simt(const AttnParams& p, cudaStream_t s);
