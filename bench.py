@@ -59,9 +59,9 @@ def parse():
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the
 # attention kernel in its current form, from one ncu capture of 8 of the 32
-# heads of t2v_5.17s (1.6524 GB), scaled by the units processed (x4) to the
+# heads of t2v_5.17s (1.6768 GB), scaled by the units processed (x4) to the
 # full launch.  Other workloads have no capture: null.
-ATTN_TRAFFIC = {("t2v_5.17s", 32, 98): 1.6524e9 * 4}
+ATTN_TRAFFIC = {("t2v_5.17s", 32, 98): 1.6768e9 * 4}
 
 
 def peaks():
