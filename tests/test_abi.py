@@ -249,3 +249,15 @@ def test_status_strings(L):
                        (-6, "VEDA_ERR_BAD_INDEX"), (-7, "VEDA_ERR_FORMAT"), (-8, "VEDA_ERR_IO"),
                        (-99, "VEDA_ERR_UNKNOWN")]:
         assert B.status_string(code) == name
+
+
+def test_c_program_uses_the_abi(L, tmp_path):
+    """A plain C program linked against libveda.so: validation, sizing, status
+    strings and the selector reader, with no Python in between."""
+    exe = tmp_path / "abi_from_c"
+    src = os.path.join(ROOT, "tests", "c", "abi_from_c.c")
+    libdir = os.path.dirname(B.LIB_PATH)
+    subprocess.run(["gcc", "-std=c11", "-O1", "-I", os.path.join(ROOT, "include"), src, "-o", str(exe),
+                    "-L", libdir, "-lveda", f"-Wl,-rpath,{libdir}"], check=True)
+    res = subprocess.run([str(exe), str(tmp_path / "sel.safetensors")], capture_output=True, text=True)
+    assert res.returncode == 0 and res.stdout.strip() == "ok", res.stderr
