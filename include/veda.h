@@ -162,7 +162,12 @@ VEDA_API veda_status veda_block_sparse_attn(const veda_problem* p, const int32_t
  *            aligned; n_rows in [1, 2^30]
  *   out      [B, n_rows, H, d] problem dtype (16-byte aligned); lse
  *            [B, H, n_rows] fp32 or NULL
- *   ws       a workspace of this problem (only its status word is used).
+ *   ws       a workspace of this problem: its status word takes device-side
+ *            errors, and with few (b, h, query tile) units the key lists are
+ *            split over several CTAs and the ranges' partial results are kept
+ *            in the workspace's scratch (overwriting what a selection call
+ *            left there) before one merge; a workspace too small for them
+ *            just runs unsplit.  Do not share it with a call in flight.
  * Errors: VEDA_ERR_INVALID_ARG for a bad pointer, stride or row count, as
  * for the other calls; device-side errors go to the status word. */
 VEDA_API veda_status veda_dense_query_attn(const veda_problem* p, const void* q_rows, int64_t n_rows,
