@@ -58,6 +58,16 @@ def test_host_call_matches_device_call(dev, name):
     assert run_both(w, inp, dev, [1, 3, 4, 16]) == [1, 3, 4, 16]
 
 
+def test_host_call_batch_two(dev):
+    """B = 2 with a reference segment: the head-range copies of every batch
+    entry land in the right place, in and out."""
+    w = REDUCED["r2va_ragged"]()
+    w = workloads.small(w.name, **{**{f: getattr(w, f) for f in ("frames", "Y", "X", "dense", "budget_video",
+                                                                  "ref_frames", "budget_ref")}, "H": 3, "B": 2})
+    inp = workloads.make_inputs(w)
+    assert run_both(w, inp, dev, [1, 2]) == [1, 2]
+
+
 def test_host_call_full_size(dev):
     w = workloads.get("t2v_5.17s")
     inp = {k: v.cpu() for k, v in workloads.make_inputs(w, device=dev).items()}
