@@ -14,6 +14,7 @@ and every full-size workload with selection checked on all rows and
 attention on a seeded sample of (b, h, query tile) units.
 """
 import math
+import warnings
 
 import numpy as np
 import pytest
@@ -21,8 +22,8 @@ import torch
 
 import learned_block_sparse_pool_b200 as veda
 import workloads
-from parity import (assert_close, assert_projection_within_bound, assert_selection, compare_selection,
-                    gather_lse, gather_units)
+from parity import (TieBandReport, assert_close, assert_projection_within_bound, assert_selection,
+                    compare_selection, gather_lse, gather_units)
 
 pytestmark = pytest.mark.gpu
 
@@ -329,6 +330,12 @@ VARIANTS = ["t2v_5.17s_k16", "t2v_5.17s_k32", "t2v_5.17s_k64", "r2va_5.17s_1x1",
             "r2va_10.13s", "r2va_14.38s"]
 
 
+def _report(name, rep):
+    """Durable per-workload tie-band report (shown in pytest's warnings summary)."""
+    warnings.warn(f"{name}: {rep.rows} selection rows, {len(rep.tie_band)} differ from the oracle only inside "
+                  f"the tie band", TieBandReport)
+
+
 @pytest.mark.parametrize("name", FULL + VARIANTS)
 def test_full_size_workload(dev, oracle_mod, name):
     w = workloads.get(name)
@@ -340,7 +347,38 @@ def test_full_size_workload(dev, oracle_mod, name):
     host = {k: v.cpu() for k, v in g.items()}
     sel = oracle_mod.select_tiles(host, w.T, w.budget_video, w.budget_ref if w.ref_frames else 0)
     rep = check_selection(oracle_mod, p, ws, iv, ir, sel, name, host)
-    print(f"{name}: {rep.rows} selection rows, {len(rep.tie_band)} inside the tie band")
+    _report(name, rep)
     units = sample_units(w, n_units=64 if name in FULL else 24)
     _, err = check_attention(oracle_mod, w, host, p, ws, sel, units, name)
     print(f"{name}: attention on {len(units)} units: max-abs {err[0]:.3g} rel-L2 {err[1]:.3g}")
+
+
+# The 14.38 s clip's budget sweep (80 / 90 / 98 % sparsity; 95 % is the
+# workload's own budget above) and the portrait clip's dense denominator
+# (budget = every tile): selection on every row, attention on sampled units
+# including the last (padded) query tile.
+SWEEP = [("t2v_14.38s", (549, 275, 55)), ("portrait_10.13s", (1922,))]
+
+
+@pytest.mark.parametrize("name,budgets", SWEEP, ids=[n for n, _ in SWEEP])
+def test_full_size_budget_sweep(dev, oracle_mod, name, budgets):
+    w0 = workloads.get(name)
+    g = workloads.make_inputs(w0, device=dev)
+    host = {k: v.cpu() for k, v in g.items()}
+    qhat = oracle_mod.project(oracle_mod.pool(host["q"], w0.T), host["w_q"])
+    khat = oracle_mod.project(oracle_mod.pool(host["k"], w0.T), host["w_k"])
+    for k in budgets:
+        w = w0.with_budget(k)
+        p = make_problem(w, g)
+        ws = veda.workspace(p)
+        iv, ir = gpu_select(p, g, ws)
+        torch.cuda.synchronize()
+        idx, kth, nxt = oracle_mod.select(qhat, khat, k)
+        sel = {"qhat": qhat, "khat": khat, "idx_v": idx, "kth_v": kth, "next_v": nxt}
+        rep = check_selection(oracle_mod, p, ws, iv, ir, sel, f"{name} k={k}", host)
+        _report(f"{name} k={k}", rep)
+        units = sample_units(w, n_units=24, seed=k)
+        _, err = check_attention(oracle_mod, w, host, p, ws, sel, units, f"{name} k={k}")
+        print(f"{name} k={k}: attention on {len(units)} units: max-abs {err[0]:.3g} rel-L2 {err[1]:.3g}")
+        del ws, iv, ir
+        torch.cuda.empty_cache()

@@ -1,9 +1,10 @@
 """The oracle pins must catch plausible mistakes.
 
-Each case copies oracle/veda_oracle.c, plants one mistake (a dropped term, a
-wrong index, a reversed comparison, ...), compiles the copy on the CPU and runs
-the pin suite against it: the suite has to fail.  The committed oracle is
-never modified.
+Each case copies the oracle (oracle/veda_oracle.c, or the Python package that
+composes its steps, oracle/__init__.py), plants one mistake (a dropped term, a
+wrong index, a reversed comparison, a swapped operand, ...), builds the copy on
+the CPU and runs the pin suite against it: the suite has to fail.  The
+committed oracle is never modified.
 """
 import os
 import subprocess
@@ -13,6 +14,7 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "veda_oracle.c")
+PY = os.path.join(ROOT, "oracle", "__init__.py")
 
 MUTANTS = {
     "pool_divides_by_T": ("o[e] = o[e] / (double)c;", "o[e] = o[e] / (double)T;"),
@@ -50,6 +52,40 @@ def test_pins_catch_planted_mistake(name, tmp_path):
     subprocess.run(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-ffp-contract=off",
                     "-o", str(so), str(mutant), "-lm"], check=True)
     env = dict(os.environ, VEDA_ORACLE_LIB=str(so), OMP_NUM_THREADS="2")
+    res = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                          os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                         cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert res.returncode != 0, f"pins did not catch mutant {name}:\n{res.stdout[-2000:]}"
+
+
+# Mistakes in the Python composition of the steps (oracle/__init__.py).
+PY_MUTANTS = {
+    "select_tiles_reference_projected_with_wq": (
+        'khat_r = project(pool(inp["k_ref"], T), inp["w_k"])',
+        'khat_r = project(pool(inp["k_ref"], T), inp["w_q"])'),
+    "select_tiles_reference_against_video_khat": (
+        'select(qhat, khat_r, budget_ref)', 'select(qhat, khat, budget_ref)'),
+    "select_tiles_reference_with_video_budget": (
+        'select(qhat, khat_r, budget_ref)', 'select(qhat, khat_r, budget_video)'),
+}
+
+
+@pytest.mark.parametrize("name", sorted(PY_MUTANTS))
+def test_pins_catch_planted_mistake_in_composition(name, tmp_path):
+    old, new = PY_MUTANTS[name]
+    src = open(PY).read()
+    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    pkg = tmp_path / "oracle"
+    pkg.mkdir()
+    (pkg / "__init__.py").write_text(src.replace(old, new))
+    (pkg / "veda_oracle.c").write_text(open(SRC).read())
+    # tests/conftest.py puts VEDA_ORACLE_DIR ahead of the repository on sys.path
+    env = dict(os.environ, VEDA_ORACLE_DIR=str(tmp_path), OMP_NUM_THREADS="2")
+    env.pop("VEDA_ORACLE_LIB", None)
+    probe = subprocess.run([sys.executable, "-c", "import sys; sys.path.insert(0, %r); "
+                            "sys.path.insert(0, %r); import oracle; print(oracle.__file__)" % (ROOT, str(tmp_path))],
+                           cwd=ROOT, env=env, capture_output=True, text=True, check=True)
+    assert probe.stdout.strip().startswith(str(tmp_path)), probe.stdout
     res = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
                           os.path.join(ROOT, "tests", "test_oracle_pins.py")],
                          cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)

@@ -421,3 +421,45 @@ def test_tiny_workload_selection_shape_and_budget(oracle_mod):
     idx = sel["idx_v"]
     assert idx.shape == (1, 2, 64, 8)
     assert (np.diff(idx, axis=-1) > 0).all() and idx.min() >= 0 and idx.max() < 64
+
+
+def test_select_tiles_reference_segment_hand_case(oracle_mod):
+    """The reference segment's key tiles are projected with W_k (the same key
+    projection as the video tiles) and ranked against the query tiles'
+    qhat independently of the video tiles, with their own budget (veyrul.com,
+    "Veda R2VA for MiniMax-H3", second paragraph: reference and video tiles
+    are selected independently with fixed budgets).
+
+    Hand derivation (d = r = 2, T = 2, every token of a tile equal, so the
+    pooled vector is that token):
+      W_q = [[1, 0], [0, 2]]  ->  qhat = pooled q W_q;  W_k = [[0, 1], [1, 0]]
+      (swaps the two channels).
+      query tile: (1, 1) -> qhat = (1, 2).
+      video tiles  (0, 5), (1, 0), (2, 2) -> khat (5, 0), (0, 1), (2, 2)
+                   -> scores 5, 2, 6 -> budget 1 keeps {2}.
+      reference    (3, 0), (0, 2), (1, 1) -> khat (0, 3), (2, 0), (1, 1)
+                   -> scores 6, 2, 3 -> budget 2 keeps {0, 2}.
+    Projecting the reference with W_q instead would give khat (3, 0), (0, 4),
+    (1, 2) and scores 3, 8, 5 (keeps {1, 2}); ranking the reference against
+    the video's khat, or with the video's budget, gives {0, 2} -> [2] or [0]."""
+    T = 2
+
+    def tiles(vals):
+        rows = []
+        for v in vals:
+            rows += [v] * T
+        return _bnhd(rows)
+
+    inp = {
+        "q": tiles([(1, 1)]),
+        "k": tiles([(0, 5), (1, 0), (2, 2)]),
+        "k_ref": tiles([(3, 0), (0, 2), (1, 1)]),
+        "w_q": torch.tensor([[[1.0, 0.0], [0.0, 2.0]]]),
+        "w_k": torch.tensor([[[0.0, 1.0], [1.0, 0.0]]]),
+    }
+    sel = oracle_mod.select_tiles(inp, T, 1, 2)
+    np.testing.assert_array_equal(sel["qhat"].reshape(-1), [1.0, 2.0])
+    np.testing.assert_array_equal(sel["khat_r"].reshape(3, 2), [[0, 3], [2, 0], [1, 1]])
+    assert sel["idx_v"].reshape(-1).tolist() == [2]
+    assert sel["idx_r"].reshape(-1).tolist() == [0, 2]
+    assert sel["kth_r"].item() == 3.0 and sel["next_r"].item() == 2.0
