@@ -26,8 +26,10 @@
  *
  * Conventions (all entry points):
  *   - Every pointer argument except `ws` sizes is a DEVICE pointer owned by
- *     the caller; the library allocates no device memory and keeps no mutable
- *     global state, so concurrent calls on different workspaces are safe.
+ *     the caller; the library allocates no device memory, and its only global
+ *     state is per device and context (the streams and events that
+ *     veda_attn_host reuses, the static array of veda_select_tiles_noalloc),
+ *     so concurrent calls on different workspaces are safe.
  *   - All work is enqueued on `stream` (a cudaStream_t; NULL = the legacy
  *     default stream); calls return after enqueueing, without synchronising.
  *   - Argument errors are detected on the host before anything is launched
@@ -180,7 +182,9 @@ VEDA_API veda_status veda_dense_query_attn(const veda_problem* p, const void* q_
  * copied in and the previous group's output, LSE and kept tiles are copied
  * out, on three streams forked from and joined back to `stream` (each head
  * is independent of the others, so a group is a complete problem of its
- * own).  Results equal veda_attn's.
+ * own).  Results equal veda_attn's.  The three streams and their events are
+ * made once per device (and again after a device reset) and reused by every
+ * call; concurrent calls on one device enqueue in turn on them.
  *   p              the problem with HOST pointers; Q and every segment packed
  *                  [B, n, H, d] (stride_h = d, stride_tok = H d, stride_b =
  *                  n H d); page-locked host memory lets the copies overlap
@@ -232,11 +236,16 @@ VEDA_API veda_status veda_topk_tiles(const veda_problem* p, int32_t* idx_video, 
  *   where the scores of a single head do not fit (about 4000 key tiles at
  *   r = 64) returns VEDA_ERR_WORKSPACE without launching anything.
  *   The call allocates nothing.  Its first call on each device looks up the
- *   array's device address (cudaGetSymbolAddress), so make that first call
- *   before capturing the stream into a CUDA graph.  All calls share the one
- *   array, which keeps the last call's contents: calls that can overlap on
- *   the GPU (different streams without ordering) race with each other;
- *   calls on one stream are ordered and safe.
+ *   array's device address (cudaGetSymbolAddress) and caches it under the
+ *   current context's id, so make that first call before capturing the
+ *   stream into a CUDA graph; after cudaDeviceReset (or any new context on
+ *   the device) the next call looks the address up again, and a failed
+ *   lookup is retried on the next call.  All calls share the one array,
+ *   which keeps the last call's contents: calls that can overlap on the GPU
+ *   (different streams without ordering) race with each other; calls on one
+ *   stream are ordered and safe.  Errors are reported through the return
+ *   code only (these selection kernels record no device-side errors, and
+ *   there is no workspace status word to read).
  *   Arguments as for veda_select_tiles(), without ws / ws_bytes. */
 VEDA_API veda_status veda_select_tiles_noalloc(const veda_problem* p, const void* w_q, const void* w_k,
                                                int32_t* idx_video, int32_t* idx_ref, veda_stream_t stream);

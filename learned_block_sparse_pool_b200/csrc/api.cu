@@ -2,12 +2,47 @@
 //
 // Every check here runs on the host before anything is enqueued, so an
 // invalid call returns an error code and leaves the device untouched.
+#include <cuda.h>
 #include <math.h>
 #include <string.h>
+
+#include <mutex>
 
 #include "veda_internal.cuh"
 
 namespace veda {
+
+namespace {
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+template <typename Fn>
+Fn driver_fn(const char* name)
+{
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint(name, &fn, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+        return nullptr;
+    return reinterpret_cast<Fn>(fn);
+}
+}  // namespace
+
+cudaError_t current_context(int* device, unsigned long long* ctx_id)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    // since CUDA 12, cudaSetDevice initialises the primary context (no-op when current)
+    if ((e = cudaSetDevice(dev)) != cudaSuccess) return e;
+    static CtxGetCurrentFn get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+    static CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+    if (!get_current || !get_id) return cudaErrorNotSupported;
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, ctx_id) != CUDA_SUCCESS)
+        return cudaErrorDeviceUninitialized;
+    *device = dev;
+    return cudaSuccess;
+}
 
 int num_sms()
 {
@@ -361,6 +396,52 @@ HostSlot host_slot(const veda_problem& p, int hc)
     return S;
 }
 
+// The three streams and nine events veda_attn_host forks its work onto, made
+// once per device and context and reused by every call (a call holds the
+// device's lock while it enqueues, so concurrent calls take turns on them).
+constexpr int kMaxDevices = 64;
+struct HostStreams {
+    std::mutex mu;
+    bool have = false;
+    unsigned long long ctx_id = 0;
+    cudaStream_t s[3] = {};
+    cudaEvent_t ev[9] = {};
+};
+HostStreams g_host_streams[kMaxDevices];
+
+// Locks and returns the device's streams and events, making them if this
+// context has none yet.  nullptr on failure (nothing locked).
+HostStreams* host_streams(std::unique_lock<std::mutex>* lock)
+{
+    int dev = 0;
+    unsigned long long id = 0;
+    if (current_context(&dev, &id) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    HostStreams& h = g_host_streams[dev];
+    std::unique_lock<std::mutex> lk(h.mu);
+    if (!h.have || h.ctx_id != id) {
+        // a new context: the previous one's handles died with it
+        HostStreams fresh_handles;
+        bool ok = true;
+        for (int i = 0; i < 3 && ok; ++i)
+            ok = cudaStreamCreateWithFlags(&fresh_handles.s[i], cudaStreamNonBlocking) == cudaSuccess;
+        for (int i = 0; i < 9 && ok; ++i)
+            ok = cudaEventCreateWithFlags(&fresh_handles.ev[i], cudaEventDisableTiming) == cudaSuccess;
+        if (!ok) {
+            for (int i = 0; i < 9; ++i)
+                if (fresh_handles.ev[i]) cudaEventDestroy(fresh_handles.ev[i]);
+            for (int i = 0; i < 3; ++i)
+                if (fresh_handles.s[i]) cudaStreamDestroy(fresh_handles.s[i]);
+            return nullptr;
+        }
+        for (int i = 0; i < 3; ++i) h.s[i] = fresh_handles.s[i];
+        for (int i = 0; i < 9; ++i) h.ev[i] = fresh_handles.ev[i];
+        h.ctx_id = id;
+        h.have = true;
+    }
+    *lock = std::move(lk);
+    return &h;
+}
+
 veda_status check_host_problem(const veda_problem& p, int heads_per_group)
 {
     if (heads_per_group < 1) return VEDA_ERR_INVALID_ARG;
@@ -492,20 +573,20 @@ veda_status veda_attn_host(const veda_problem* p, const void* w_q, const void* w
     cudaStream_t caller = (cudaStream_t)stream;
 
     // three streams (copy in, compute, copy out) forked from and joined back to the caller's stream
-    cudaStream_t sin = nullptr, scomp = nullptr, sout = nullptr;
-    cudaEvent_t ev[9] = {};
-    bool ok = cudaStreamCreateWithFlags(&sin, cudaStreamNonBlocking) == cudaSuccess &&
-              cudaStreamCreateWithFlags(&scomp, cudaStreamNonBlocking) == cudaSuccess &&
-              cudaStreamCreateWithFlags(&sout, cudaStreamNonBlocking) == cudaSuccess;
-    for (int i = 0; i < 9 && ok; ++i) ok = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) == cudaSuccess;
+    std::unique_lock<std::mutex> hs_lock;
+    HostStreams* hs = host_streams(&hs_lock);
+    if (!hs) return VEDA_ERR_CUDA;
+    cudaStream_t sin = hs->s[0], scomp = hs->s[1], sout = hs->s[2];
+    cudaEvent_t* ev = hs->ev;
     cudaEvent_t &e_fork = ev[0], &e_in0 = ev[1], &e_in1 = ev[2], &e_c0 = ev[3], &e_c1 = ev[4], &e_free0 = ev[5],
                 &e_free1 = ev[6], &e_comp_end = ev[7], &e_out_end = ev[8];
     cudaEvent_t e_in[2] = {e_in0, e_in1}, e_comp[2] = {e_c0, e_c1}, e_free[2] = {e_free0, e_free1};
-    st = ok ? VEDA_OK : VEDA_ERR_CUDA;
-    if (st == VEDA_OK) {
-        ok = cudaEventRecord(e_fork, caller) == cudaSuccess && cudaStreamWaitEvent(sin, e_fork, 0) == cudaSuccess &&
-             cudaStreamWaitEvent(scomp, e_fork, 0) == cudaSuccess &&
-             cudaStreamWaitEvent(sout, e_fork, 0) == cudaSuccess;
+    st = VEDA_OK;
+    {
+        const bool ok = cudaEventRecord(e_fork, caller) == cudaSuccess &&
+                        cudaStreamWaitEvent(sin, e_fork, 0) == cudaSuccess &&
+                        cudaStreamWaitEvent(scomp, e_fork, 0) == cudaSuccess &&
+                        cudaStreamWaitEvent(sout, e_fork, 0) == cudaSuccess;
         if (!ok) st = VEDA_ERR_CUDA;
     }
     const veda_segment* hsegs[3] = {&P.video, &P.ref, &P.dense};
@@ -579,19 +660,13 @@ veda_status veda_attn_host(const veda_problem* p, const void* w_q, const void* w
         if (!k_ok) st = VEDA_ERR_CUDA;
     }
     // join: the caller's stream waits for every copy and kernel of this call
-    if (sin && scomp && sout && ev[7] && ev[8]) {
-        cudaEventRecord(e_comp_end, scomp);
-        cudaEventRecord(e_out_end, sout);
-        cudaStreamWaitEvent(caller, e_comp_end, 0);
-        cudaStreamWaitEvent(caller, e_out_end, 0);
-        cudaEventRecord(e_fork, sin);               // the copy-in stream's last work
-        cudaStreamWaitEvent(caller, e_fork, 0);
-    }
-    for (int i = 0; i < 9; ++i)
-        if (ev[i]) cudaEventDestroy(ev[i]);         // released once their work completes
-    if (sin) cudaStreamDestroy(sin);
-    if (scomp) cudaStreamDestroy(scomp);
-    if (sout) cudaStreamDestroy(sout);
+    // (the join is enqueued on every path, so no stream is left forked)
+    cudaEventRecord(e_comp_end, scomp);
+    cudaEventRecord(e_out_end, sout);
+    cudaStreamWaitEvent(caller, e_comp_end, 0);
+    cudaStreamWaitEvent(caller, e_out_end, 0);
+    cudaEventRecord(e_fork, sin);               // the copy-in stream's last work
+    cudaStreamWaitEvent(caller, e_fork, 0);
     return st;
 }
 

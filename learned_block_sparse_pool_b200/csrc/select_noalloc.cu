@@ -26,23 +26,38 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
-// Device address of g_scratch, resolved once per device (the name itself is
-// only a host-side stand-in and must never be passed to a kernel).
-std::once_flag g_once[kMaxDevices];
-void* g_addr[kMaxDevices];
-cudaError_t g_addr_err[kMaxDevices];
+// Device address of g_scratch in the current context.  The name g_scratch is
+// only a host-side stand-in and must never be passed to a kernel; the device
+// address is looked up with cudaGetSymbolAddress once per context and cached
+// under the context's unique id, so a context that is destroyed and created
+// again (cudaDeviceReset, or the primary context released and retained
+// again) gets a fresh lookup instead of a stale address.  A failed lookup is
+// not cached: the next call tries again.
+struct ScratchCache {
+    std::mutex mu;
+    bool have = false;
+    unsigned long long ctx_id = 0;
+    void* addr = nullptr;
+};
+ScratchCache g_cache[kMaxDevices];
 
 cudaError_t scratch_address(void** out)
 {
     int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    unsigned long long id = 0;
+    cudaError_t e = current_context(&dev, &id);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::call_once(g_once[dev], [dev] {
-        g_addr_err[dev] = cudaGetSymbolAddress(&g_addr[dev], g_scratch);
-    });
-    if (g_addr_err[dev] != cudaSuccess) return g_addr_err[dev];
-    *out = g_addr[dev];
+    ScratchCache& c = g_cache[dev];
+    std::lock_guard<std::mutex> lock(c.mu);
+    if (!c.have || c.ctx_id != id) {
+        void* a = nullptr;
+        if ((e = cudaGetSymbolAddress(&a, g_scratch)) != cudaSuccess) return e;
+        c.addr = a;
+        c.ctx_id = id;
+        c.have = true;
+    }
+    *out = c.addr;
     return cudaSuccess;
 }
 
@@ -69,7 +84,7 @@ extern "C" VEDA_API veda_status veda_select_tiles_noalloc(const veda_problem* p,
     // scratch needed by one head: qhat, khat, khat_ref, scores, scores_ref
     const int64_t ld_v = cdiv(nq, 32) * 32, ld_r = cdiv(nr, 32) * 32;
     const size_t per_head = sizeof(float) * (size_t)(2 * nq * p->r + nr * p->r + nq * ld_v + nq * ld_r);
-    const size_t fixed = kAlignBytes /* status word */ + 5 * kAlignBytes /* region padding */;
+    const size_t fixed = kAlignBytes /* unused head block */ + 5 * kAlignBytes /* region padding */;
     if (per_head + fixed > kScratchBytes) return VEDA_ERR_WORKSPACE;   // one head does not fit
     const int hc_max = (int)std::min<size_t>((size_t)p->H, (kScratchBytes - fixed) / per_head);
 
@@ -77,8 +92,6 @@ extern "C" VEDA_API veda_status veda_select_tiles_noalloc(const veda_problem* p,
     if (scratch_address(&base) != cudaSuccess) return VEDA_ERR_CUDA;
     cudaStream_t s = (cudaStream_t)stream;
     char* sb = static_cast<char*>(base);
-    uint32_t* status = reinterpret_cast<uint32_t*>(sb);
-    if (cudaMemsetAsync(status, 0, sizeof(uint32_t), s) != cudaSuccess) return VEDA_ERR_CUDA;
 
     const size_t es = p->dtype == VEDA_BF16 ? 2 : 4;
     const char* wq = static_cast<const char*>(w_q);
@@ -128,7 +141,7 @@ extern "C" VEDA_API veda_status veda_select_tiles_noalloc(const veda_problem* p,
 
             const int64_t row0 = ((int64_t)b * p->H + h0) * nq;
             TopkParams T{};
-            T.status = status;
+            T.status = nullptr;     // the selection kernels record no device-side errors
             T.rows = (int64_t)hc * nq;
             T.scores = sc_v; T.ld = ld_v; T.n = (int32_t)nq; T.k = p->video.budget;
             T.idx = idx_video + row0 * p->video.budget;

@@ -98,4 +98,11 @@ cudaError_t launch_attn_simt(const AttnParams& p, cudaStream_t s);
 
 int num_sms();
 
+// The current device and a process-unique id of its current CUDA context
+// (the device's primary context is made current first).  Host-side caches of
+// per-context objects (a symbol's device address, streams, events) are keyed
+// by this id, so a context that is destroyed and created again (for example
+// by cudaDeviceReset) gets fresh objects.
+cudaError_t current_context(int* device, unsigned long long* ctx_id);
+
 }  // namespace veda

@@ -5,6 +5,7 @@ import ctypes
 import os
 import re
 import subprocess
+import sys
 
 import pytest
 
@@ -261,3 +262,32 @@ def test_c_program_uses_the_abi(L, tmp_path):
                     "-L", libdir, "-lveda", f"-Wl,-rpath,{libdir}"], check=True)
     res = subprocess.run([str(exe), str(tmp_path / "sel.safetensors")], capture_output=True, text=True)
     assert res.returncode == 0 and res.stdout.strip() == "ok", res.stderr
+
+
+NOALLOC_REJECT = r"""
+import ctypes, sys
+sys.path.insert(0, %r)
+import learned_block_sparse_pool_b200 as veda
+from learned_block_sparse_pool_b200 import binding as B
+p = B.veda_problem()
+p.B, p.H, p.d, p.tile, p.r = 1, 1, 128, 128, 64
+p.dtype = B.VEDA_BF16
+n = 4096 * 128                                    # 4096 key tiles: one head's scores exceed 64 MiB
+p.q = 0x100000
+p.q_stride_b, p.q_stride_tok, p.q_stride_h = n * 128, 128, 128
+p.video.k, p.video.v = 0x200000, 0x300000
+p.video.n_tokens = n
+p.video.stride_b, p.video.stride_tok, p.video.stride_h = n * 128, 128, 128
+p.video.budget = 8
+print(veda.lib().veda_select_tiles_noalloc(ctypes.byref(p), 0x400000, 0x500000, 0x600000, None, None))
+"""
+
+
+def test_noalloc_rejects_a_head_that_does_not_fit_without_a_device(L):
+    """The static scratch array holds 64 MiB; a single head with 4096 key
+    tiles needs more, and the call must refuse it on the host.  Run with no
+    device visible, so the fake pointers can never reach a kernel."""
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    res = subprocess.run([sys.executable, "-c", NOALLOC_REJECT % ROOT], env=env, capture_output=True, text=True,
+                         check=True, timeout=300)
+    assert int(res.stdout.strip().splitlines()[-1]) == B.VEDA_ERR_WORKSPACE

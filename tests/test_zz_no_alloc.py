@@ -7,10 +7,10 @@ array inside the library, so the caller passes only inputs and outputs.
 Checked through the C ABI against veda_select_tiles (the workspace entry
 point): the kept tiles must be identical, on two calls in a row (the static
 array keeps the previous call's contents, which must not leak into the next
-result).  This file is collected last on purpose.
+result).  pytest collects this file last (its name sorts last), so a run that
+stops at the first failure has run every other test before this one; the
+tests pass either way, alone in a fresh process or after the others.
 """
-import ctypes
-
 import pytest
 import torch
 
@@ -56,8 +56,9 @@ def _compare_two_calls(w, g):
 
 
 def test_noalloc_matches_workspace_entry_full_clip(dev):
-    """5.17 s clip (32 heads, 977 tiles): the static array holds 14 heads'
-    scores, so the call runs in three head groups."""
+    """5.17 s clip (32 heads, 977 tiles): one head needs 4,376,960 bytes of
+    scratch (q-hat, k-hat and the 977 x 992 score rows), so the 64 MiB array
+    holds 15 heads and the call runs in three head groups (15 + 15 + 2)."""
     w = workloads.get("t2v_5.17s")
     _compare_two_calls(w, workloads.make_inputs(w, device=dev))
 
@@ -69,16 +70,17 @@ def test_noalloc_matches_workspace_entry_batch_and_reference(dev):
 
 
 def test_noalloc_rejects_a_head_that_does_not_fit(dev):
-    """4096 key tiles: one head's scores alone exceed the static array."""
-    p = B.veda_problem()
-    p.B, p.H, p.d, p.tile, p.r = 1, 1, 128, 128, 64
-    p.dtype = B.VEDA_BF16
+    """4096 key tiles: one head's scores alone exceed the static array, so the
+    call returns VEDA_ERR_WORKSPACE before launching anything.  The problem
+    points at real device tensors of its full size, so even a call that went
+    further would read valid memory."""
     n = 4096 * 128
-    p.q = 0x100000
-    p.q_stride_b, p.q_stride_tok, p.q_stride_h = n * 128, 128, 128
-    p.video.k, p.video.v = 0x200000, 0x300000
-    p.video.n_tokens = n
-    p.video.stride_b, p.video.stride_tok, p.video.stride_h = n * 128, 128, 128
-    p.video.budget = 8
-    st = veda.lib().veda_select_tiles_noalloc(ctypes.byref(p), 0x400000, 0x500000, 0x600000, None, None)
+    q = torch.zeros((1, n, 1, 128), dtype=torch.bfloat16, device=dev)
+    k = torch.zeros_like(q)
+    v = torch.zeros_like(q)
+    w = torch.zeros((1, 128, 64), dtype=torch.bfloat16, device=dev)
+    p = veda.Problem(q, k, v, tile=128, r=64, budget=8)
+    iv, _ = veda.alloc_indices(p)
+    st = veda.lib().veda_select_tiles_noalloc(p.ref(), w.data_ptr(), w.data_ptr(), iv.data_ptr(), None,
+                                              torch.cuda.current_stream().cuda_stream)
     assert st == B.VEDA_ERR_WORKSPACE
