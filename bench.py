@@ -2,9 +2,9 @@
 """Benchmark of the Veda-style block-sparse attention hot path on B200.
 
 One step = one full pass of the path over one synthetic layer call:
-tile pool + selector projection -> tile scores -> fixed-budget top-k ->
-block-sparse attention (the four stages veda_attn runs), inputs resident in
-HBM.  Default workload: the 1344x768, 24 fps, 5.17 s landscape clip
+tile pool + selector projection -> tile scores + fixed-budget top-k (fused on
+the tensor cores) -> block-sparse attention (the stages veda_attn runs),
+inputs resident in HBM.  Default workload: the 1344x768, 24 fps, 5.17 s landscape clip
 (31 x 48 x 84 = 124,992 video tokens, 32 heads, head dim 128, tile 128,
 90% sparsity = 98 kept tiles, 512 text + 256 audio dense keys), bf16.
 
@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--budget", type=int, default=0, help="override the video budget")
     ap.add_argument("--heads", type=int, default=0, help="override the head count (smaller profiling cases)")
     ap.add_argument("--simt", action="store_true", help="use the SIMT attention kernel")
+    ap.add_argument("--unfused-selection", action="store_true",
+                    help="time the three-kernel selection (fp32 SIMT scores, then the warp-per-row top-k)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ncu", action="store_true", help="short run for profiler captures (no extras)")
@@ -262,18 +264,24 @@ def main():
     out, _ = veda.alloc_output(p)
     stream = torch.cuda.current_stream(dev)
 
+    # the stages of one call, each bracketed by CUDA events on the launching stream
+    if args.unfused_selection:
+        stages = [("pool_project", lambda: veda.pool_project(p, g["w_q"], g["w_k"], ws, stream)),
+                  ("score", lambda: veda.score_tiles(p, ws, stream)),
+                  ("topk", lambda: veda.topk_tiles(p, iv, ir, ws, stream))]
+    else:
+        stages = [("pool_project", lambda: veda.pool_project(p, g["w_q"], g["w_k"], ws, stream)),
+                  ("select", lambda: veda.score_topk_tiles(p, iv, ir, ws, stream))]
+    stages.append(("attention", lambda: veda.block_sparse_attn(p, iv, ir, out, None, ws, stream)))
+    n_st = len(stages)
+
     def step(ev):
-        veda.pool_project(p, g["w_q"], g["w_k"], ws, stream)
-        ev[1].record(stream)
-        veda.score_tiles(p, ws, stream)
-        ev[2].record(stream)
-        veda.topk_tiles(p, iv, ir, ws, stream)
-        ev[3].record(stream)
-        veda.block_sparse_attn(p, iv, ir, out, None, ws, stream)
-        ev[4].record(stream)
+        for s_i, (_, fn) in enumerate(stages):
+            fn()
+            ev[s_i + 1].record(stream)
 
     def events():
-        return [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        return [torch.cuda.Event(enable_timing=True) for _ in range(n_st + 1)]
 
     clocks = ClockSampler(local)
     clocks.start()
@@ -306,12 +314,13 @@ def main():
         raise RuntimeError(f"device status after timing: {veda.status_string(st)}")
 
     total_ms = t_start.elapsed_time(t_end)
-    stage = [[evs[k][s].elapsed_time(evs[k][s + 1]) for k in range(args.steps)] for s in range(4)]
+    stage = [[evs[k][s].elapsed_time(evs[k][s + 1]) for k in range(args.steps)] for s in range(n_st)]
     stage_avg = [sum(x) / len(x) for x in stage]
     total_ms, *stage_avg = max_over_ranks(dist, [total_ms] + stage_avg, dev)
+    st_ms = {name: stage_avg[i] for i, (name, _) in enumerate(stages)}
 
     pk, pk_src = peaks()
-    attn_s = stage_avg[3] / 1e3
+    attn_s = st_ms["attention"] / 1e3
     flops = w.kept_flops()
     achieved_tf = flops / attn_s / 1e12
     sustained_tf = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
@@ -324,11 +333,35 @@ def main():
     esz = 2 if w.dtype == "bf16" else 4
     pool_bytes = (2 * w.n_video + w.n_ref) * w.B * w.H * w.d * esz
     rows = w.B * w.H * w.n_q_tiles
-    # a row's scores are read unless every tile is kept; the kept indices are written
-    topk_bytes = rows * ((w.n_q_tiles * 4 if w.budget_video < w.n_q_tiles else 0) + w.budget_video * 4)
-    if w.ref_frames:
-        topk_bytes += rows * ((w.n_ref_tiles * 4 if w.budget_ref < w.n_ref_tiles else 0) + w.budget_ref * 4)
-    launches_per_step = 4 + (2 if w.ref_frames else 0)
+    selector = {
+        "pool_project_gbs": round(pool_bytes / (st_ms["pool_project"] / 1e3) / 1e9, 1),
+        "pool_project_frac": round(pool_bytes / (st_ms["pool_project"] / 1e3) / 1e9 / hbm, 4),
+        "peak_gbs": hbm, "peak_kind": f"HBM copy ({pk_src})",
+    }
+    segs = [(w.n_q_tiles, w.budget_video)] + ([(w.n_ref_tiles, w.budget_ref)] if w.ref_frames else [])
+    score_flop = sum(2.0 * w.r * rows * nk for nk, _ in segs)
+    if args.unfused_selection:
+        # a row's scores are read unless every tile is kept; the kept indices are written
+        topk_bytes = sum(rows * ((nk * 4 if k < nk else 0) + k * 4) for nk, k in segs)
+        selector.update({
+            "topk_gbs": round(topk_bytes / (st_ms["topk"] / 1e3) / 1e9, 1),
+            "topk_frac": round(topk_bytes / (st_ms["topk"] / 1e3) / 1e9 / hbm, 4),
+            "score_kernel": "SIMT fp32 contraction (alu-bound)",
+            "score_gflops": round(score_flop / (st_ms["score"] / 1e3) / 1e9, 1),
+        })
+        launches_per_step = 2 + 2 * len(segs)
+    else:
+        # fused score + top-k: reads the bf16 projection planes (k-hat from L2)
+        # and writes the kept indices; its work is the tensor-core scoring of
+        # every (query tile, key tile) pair, repeated for each pass
+        sel_bytes = sum(rows * k * 4 for _, k in segs) + 6 * 64 * rows * (1 + len(segs))
+        selector.update({
+            "select_kernel": "fused tensor-core score + on-chip top-k (no score matrix in HBM)",
+            "select_ms": round(st_ms["select"], 4),
+            "select_algorithmic_bytes": sel_bytes,
+            "select_score_gflops": round(score_flop / (st_ms["select"] / 1e3) / 1e9, 1),
+        })
+        launches_per_step = 3 + sum(1 for nk, k in segs if 128 < nk and k < nk)   # + fallback top-k
 
     res = {
         "metric": METRIC,
@@ -344,8 +377,7 @@ def main():
         "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic (seeded; N(0,1) + smooth sinusoid component, shapes of the 1344x768 24 fps clips)",
         "config": bench_config(w, n, args.simt),
-        "kernels_ms": {"pool_project": round(stage_avg[0], 4), "score": round(stage_avg[1], 4),
-                       "topk": round(stage_avg[2], 4), "attention": round(stage_avg[3], 4)},
+        "kernels_ms": {name: round(v, 4) for name, v in st_ms.items()},
         "roofline": {
             "kernel": "block-sparse attention",
             "bound": "tensor", "achieved": round(achieved_tf, 2), "peak": peak_tf, "unit": "TFLOP/s",
@@ -357,14 +389,7 @@ def main():
             "frac_of_sustained_peak": round(achieved_tf / sustained_tf, 4),
             "algorithmic": f"{flops:.4g} FLOP per launch = 4*T*T*d x kept (b,h,q-tile,k-tile) pairs",
         },
-        "selector_hbm": {
-            "pool_project_gbs": round(pool_bytes / (stage_avg[0] / 1e3) / 1e9, 1),
-            "pool_project_frac": round(pool_bytes / (stage_avg[0] / 1e3) / 1e9 / hbm, 4),
-            "topk_gbs": round(topk_bytes / (stage_avg[2] / 1e3) / 1e9, 1),
-            "topk_frac": round(topk_bytes / (stage_avg[2] / 1e3) / 1e9 / hbm, 4),
-            "peak_gbs": hbm, "peak_kind": f"HBM copy ({pk_src})",
-            "score_kernel": "SIMT fp32 contraction (alu-bound)",
-        },
+        "selector_hbm": selector,
         "clocks": clk,
         "gpu_launches": launches_per_step * args.steps,
     }

@@ -90,6 +90,13 @@ typedef enum { VEDA_F32 = 0, VEDA_BF16 = 1 } veda_dtype;
                                        reports VEDA_ERR_TIMEOUT through
                                        veda_check_status(); its output is then
                                        undefined.  No effect on other kernels. */
+#define VEDA_FLAG_UNFUSED_SELECTION 4u /* select tiles with the three-kernel path
+                                       (fp32 SIMT scores written to the
+                                       workspace, then the warp-per-row top-k)
+                                       instead of the fused tensor-core score +
+                                       top-k: a cross-check path.  The fused
+                                       path needs r <= 64 and falls back to
+                                       this one otherwise. */
 
 /* One key/value segment, [B, n_tokens, H, d] (d contiguous). */
 typedef struct {
@@ -134,7 +141,9 @@ VEDA_API veda_status veda_workspace_init(void* ws, size_t ws_bytes, veda_stream_
 
 /* Steps 1-3: pool + project Q and K, score every key tile, keep the top
  * `budget` per (b, h, query tile) for the video segment and, when present,
- * independently for the reference segment.
+ * independently for the reference segment.  Steps 2-3 run fused on the
+ * tensor cores (see veda_score_topk_tiles) unless r > 64 or
+ * VEDA_FLAG_UNFUSED_SELECTION is set.
  *   w_q, w_k   [H, d, r] device, problem dtype
  *   idx_video  [B, H, n_q_tiles, video.budget] int32 out (ascending rows)
  *   idx_ref    [B, H, n_q_tiles, ref.budget]   int32 out; NULL iff no reference */
@@ -222,6 +231,16 @@ VEDA_API veda_status veda_score_tiles(const veda_problem* p, void* ws, size_t ws
 /* Step 3: top-k of the workspace scores into idx_video / idx_ref. */
 VEDA_API veda_status veda_topk_tiles(const veda_problem* p, int32_t* idx_video, int32_t* idx_ref,
                             void* ws, size_t ws_bytes, veda_stream_t stream);
+/* Steps 2-3 fused (what veda_select_tiles runs after veda_pool_project): the
+ * tile scores are computed on the tensor cores from the projections in the
+ * workspace, as three bf16 parts per value whose six leading products give
+ * fp32 accuracy, and each row's top-k is selected on chip without writing
+ * the score matrix; rows whose on-chip selection cannot finish (a score band
+ * wider than its buffer, or a NaN) get their scores written to the
+ * workspace and go through the step-3 kernel.  With r > 64 or
+ * VEDA_FLAG_UNFUSED_SELECTION this runs steps 2 and 3 unfused. */
+VEDA_API veda_status veda_score_topk_tiles(const veda_problem* p, int32_t* idx_video, int32_t* idx_ref,
+                                           void* ws, size_t ws_bytes, veda_stream_t stream);
 
 /* Tile selection without a workspace, for callers that cannot allocate
  * device memory when they call: a serving engine that plans all memory up
@@ -229,7 +248,9 @@ VEDA_API veda_status veda_topk_tiles(const veda_problem* p, int32_t* idx_video, 
  * hook may not allocate, or a latency-critical loop that cannot afford the
  * device synchronisation cudaMalloc implies.  The pages have no counterpart
  * of this call; it exists only for such callers.
- *   Computes exactly what veda_select_tiles() computes (same kernels), with
+ *   Computes exactly what veda_select_tiles() computes with
+ *   VEDA_FLAG_UNFUSED_SELECTION (the same pool + project, fp32 score and
+ *   top-k kernels), with
  *   its scratch in a 64 MiB array that this library reserves statically on
  *   every GPU that uses it and keeps until the process exits.  The problem is
  *   processed one batch entry and one group of heads at a time; a problem
@@ -254,7 +275,10 @@ VEDA_API veda_status veda_select_tiles_noalloc(const veda_problem* p, const void
  *   which = 0: qhat [B,H,n_q_tiles,r] fp32     1: khat video [B,H,n_q_tiles,r]
  *           2: khat ref [B,H,n_ref_tiles,r]    3: scores video [B,H,n_q_tiles,ld]
  *           4: scores ref [B,H,n_q_tiles,ld]
- * *ld receives the row stride (elements) of the score matrices (>= n tiles). */
+ *           5 / 6: int32 rows the fused selection (video / reference) left
+ *              to the step-3 kernel: [0] = count, then the row ids
+ * *ld receives the row stride (elements) of the score matrices (>= n tiles;
+ * 1 for which = 5, 6). */
 VEDA_API veda_status veda_workspace_view(const veda_problem* p, void* ws, size_t ws_bytes, int which,
                                 const void** ptr, int64_t* ld);
 

@@ -8,9 +8,11 @@ ctypes marshalling layer over it.  Build the library with
 `python -m learned_block_sparse_pool_b200.build`.
 """
 from .binding import (EXPORTS, LIB_PATH, Problem, Selector, VedaError, alloc_indices, alloc_output, attn, attn_host, attn_host_buffer, dense_query_attn,
-                      block_sparse_attn, check_status, lib, pool_project, score_tiles, select_tiles,
+                      block_sparse_attn, check_status, fallback_rows, lib, pool_project, score_tiles, score_topk_tiles,
+                      select_tiles,
                       select_tiles_noalloc, status_string, topk_tiles, workspace, workspace_size, workspace_view)
 
 __all__ = ["EXPORTS", "LIB_PATH", "Problem", "Selector", "VedaError", "alloc_indices", "alloc_output", "attn", "attn_host", "attn_host_buffer", "dense_query_attn",
-           "block_sparse_attn", "check_status", "lib", "pool_project", "score_tiles", "select_tiles",
+           "block_sparse_attn", "check_status", "fallback_rows", "lib", "pool_project", "score_tiles",
+           "score_topk_tiles", "select_tiles",
            "select_tiles_noalloc", "status_string", "topk_tiles", "workspace", "workspace_size", "workspace_view"]

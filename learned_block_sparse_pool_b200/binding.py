@@ -28,13 +28,14 @@ VEDA_ERR_IO = -8
 VEDA_F32, VEDA_BF16 = 0, 1
 VEDA_FLAG_SIMT_ATTENTION = 1
 VEDA_FLAG_TEST_SHORT_WAITS = 2
+VEDA_FLAG_UNFUSED_SELECTION = 4
 
 EXPORTS = ("veda_workspace_size", "veda_workspace_init", "veda_select_tiles", "veda_block_sparse_attn",
            "veda_attn", "veda_pool_project", "veda_score_tiles", "veda_topk_tiles", "veda_workspace_view",
            "veda_check_status", "veda_status_string", "veda_select_tiles_noalloc", "veda_dense_query_attn",
            "veda_selector_open", "veda_selector_close", "veda_selector_check", "veda_selector_count",
            "veda_selector_find", "veda_selector_info", "veda_selector_metadata", "veda_selector_read",
-           "veda_attn_host_buffer_size", "veda_attn_host")
+           "veda_attn_host_buffer_size", "veda_attn_host", "veda_score_topk_tiles")
 
 
 class VedaError(RuntimeError):
@@ -80,6 +81,7 @@ def lib() -> ctypes.CDLL:
         L.veda_pool_project.argtypes = [P, vp, vp, vp, sz, vp]
         L.veda_score_tiles.argtypes = [P, vp, sz, vp]
         L.veda_topk_tiles.argtypes = [P, i32p, i32p, vp, sz, vp]
+        L.veda_score_topk_tiles.argtypes = [P, i32p, i32p, vp, sz, vp]
         L.veda_workspace_view.argtypes = [P, vp, sz, ctypes.c_int, ctypes.POINTER(ctypes.c_void_p),
                                           ctypes.POINTER(ctypes.c_int64)]
         L.veda_check_status.argtypes = [vp, vp]
@@ -274,6 +276,23 @@ def score_tiles(p: Problem, ws, stream=None) -> None:
 def topk_tiles(p: Problem, idx_v, idx_r, ws, stream=None) -> None:
     _check(lib().veda_topk_tiles(p.ref(), _ptr(idx_v), _ptr(idx_r), ws.data_ptr(), ws.numel(),
                                  _stream(stream)), "veda_topk_tiles")
+
+
+def score_topk_tiles(p: Problem, idx_v, idx_r, ws, stream=None) -> None:
+    """Steps 2-3 (fused on the tensor cores unless unsupported or flagged)."""
+    _check(lib().veda_score_topk_tiles(p.ref(), _ptr(idx_v), _ptr(idx_r), ws.data_ptr(), ws.numel(),
+                                       _stream(stream)), "veda_score_topk_tiles")
+
+
+def fallback_rows(p: Problem, ws, ref: bool = False) -> torch.Tensor:
+    """Row ids the last fused selection left to the exact step-3 kernel."""
+    ptr = ctypes.c_void_p()
+    ld = ctypes.c_int64()
+    _check(lib().veda_workspace_view(p.ref(), ws.data_ptr(), ws.numel(), 6 if ref else 5, ctypes.byref(ptr),
+                                     ctypes.byref(ld)), "veda_workspace_view")
+    off = ptr.value - ws.data_ptr()
+    count = int(ws[off:off + 4].view(torch.int32).item())
+    return ws[off + 4:off + 4 + 4 * count].view(torch.int32).clone()
 
 
 def workspace_view(p: Problem, ws, which: int) -> torch.Tensor:

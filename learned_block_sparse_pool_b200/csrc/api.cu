@@ -54,7 +54,6 @@ int num_sms()
 
 cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s);
 bool attn_tc_supported(const AttnParams& p);
-int topk_max_tiles();
 
 namespace {
 
@@ -66,8 +65,14 @@ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 struct Layout {
     int64_t nq, nr;          // query (= video key) tiles, reference tiles
     int64_t ld_v, ld_r;      // score row strides (elements)
-    size_t qhat, khat, khat_r, sc_v, sc_r, total;
+    size_t qhat, khat, khat_r, sc_v, sc_r;
+    size_t qpl, kpl, kpl_r;  // bf16 planes of the projections (fused scoring), r <= 64
+    size_t ksm, ksm_r;       // the planes of the 64 sampled key tiles per head
+    size_t fb_v, fb_r;       // fused selection: rows left to the exact top-k (count, then ids)
+    size_t total;
 };
+
+constexpr int kPlaneWidth = 64;   // columns of a projection plane row
 
 size_t esize(veda_dtype t) { return t == VEDA_BF16 ? 2 : 4; }
 
@@ -108,7 +113,8 @@ veda_status validate(const veda_problem* pp)
     if (p.tile != 64 && p.tile != 128) return VEDA_ERR_UNSUPPORTED;
     if (p.r > 128 || p.r % 4 != 0) return VEDA_ERR_UNSUPPORTED;
     if (!(p.softmax_scale >= 0.f) || !isfinite(p.softmax_scale)) return VEDA_ERR_INVALID_ARG;
-    if (p.flags & ~(VEDA_FLAG_SIMT_ATTENTION | VEDA_FLAG_TEST_SHORT_WAITS)) return VEDA_ERR_INVALID_ARG;
+    if (p.flags & ~(VEDA_FLAG_SIMT_ATTENTION | VEDA_FLAG_TEST_SHORT_WAITS | VEDA_FLAG_UNFUSED_SELECTION))
+        return VEDA_ERR_INVALID_ARG;
     if (!p.q || !aligned16(p.q)) return VEDA_ERR_INVALID_ARG;
     const size_t es = esize(p.dtype);
     if (!stride_ok(p.q_stride_b, es) || !stride_ok(p.q_stride_tok, es) || !stride_ok(p.q_stride_h, es))
@@ -134,6 +140,14 @@ Layout layout(const veda_problem& p)
     L.khat_r = off; off = align_up(off + sizeof(float) * BH * L.nr * p.r, kAlign);
     L.sc_v = off;   off = align_up(off + sizeof(float) * BH * L.nq * L.ld_v, kAlign);
     L.sc_r = off;   off = align_up(off + sizeof(float) * BH * L.nq * L.ld_r, kAlign);
+    const bool planes = p.r <= kPlaneWidth;
+    L.qpl = off;    off = align_up(off + (planes ? 3 * 2 * BH * L.nq * kPlaneWidth : 0), kAlign);
+    L.kpl = off;    off = align_up(off + (planes ? 3 * 2 * BH * L.nq * kPlaneWidth : 0), kAlign);
+    L.kpl_r = off;  off = align_up(off + (planes ? 3 * 2 * BH * L.nr * kPlaneWidth : 0), kAlign);
+    L.ksm = off;    off = align_up(off + (planes ? 3 * 2 * BH * 64 * kPlaneWidth : 0), kAlign);
+    L.ksm_r = off;  off = align_up(off + (planes && L.nr > 0 ? 3 * 2 * BH * 64 * kPlaneWidth : 0), kAlign);
+    L.fb_v = off;   off = align_up(off + sizeof(int32_t) * (1 + BH * L.nq), kAlign);
+    L.fb_r = off;   off = align_up(off + sizeof(int32_t) * (L.nr > 0 ? 1 + BH * L.nq : 0), kAlign);
     L.total = off;
     return L;
 }
@@ -172,20 +186,26 @@ veda_status do_pool_project(const veda_problem& p, const Layout& L, const void* 
     memset(&P, 0, sizeof P);
     P.B = p.B; P.H = p.H; P.d = p.d; P.T = p.tile; P.r = p.r; P.dtype = p.dtype;
     int64_t items = 0;
-    auto add = [&](const void* x, int64_t sb, int64_t st, int64_t sh, int64_t n, const void* w, float* out) {
+    const bool planes = p.r <= kPlaneWidth;   // bf16 planes for the tensor-core scoring
+    auto add = [&](const void* x, int64_t sb, int64_t st, int64_t sh, int64_t n, const void* w, float* out,
+                   size_t plane_off, size_t sample_off) {
         PoolJob& J = P.job[P.n_jobs++];
         J.x = x; J.sb = sb; J.st = st; J.sh = sh; J.n_tokens = n;
         J.n_tiles = (int32_t)ceil_div(n, p.tile);
         J.first_item = items;
         J.w = w; J.out = out;
+        J.planes = planes ? at<uint16_t>(ws, plane_off) : nullptr;
+        J.plane_stride = (int64_t)p.B * p.H * J.n_tiles * kPlaneWidth;
+        J.sample_planes = planes && sample_off ? at<uint16_t>(ws, sample_off) : nullptr;
+        J.sample_plane_stride = (int64_t)p.B * p.H * 64 * kPlaneWidth;
         items += (int64_t)p.B * p.H * J.n_tiles;
     };
-    add(p.q, p.q_stride_b, p.q_stride_tok, p.q_stride_h, p.video.n_tokens, w_q, at<float>(ws, L.qhat));
+    add(p.q, p.q_stride_b, p.q_stride_tok, p.q_stride_h, p.video.n_tokens, w_q, at<float>(ws, L.qhat), L.qpl, 0);
     add(p.video.k, p.video.stride_b, p.video.stride_tok, p.video.stride_h, p.video.n_tokens, w_k,
-        at<float>(ws, L.khat));
+        at<float>(ws, L.khat), L.kpl, L.ksm);
     if (p.ref.n_tokens > 0)
         add(p.ref.k, p.ref.stride_b, p.ref.stride_tok, p.ref.stride_h, p.ref.n_tokens, w_k,
-            at<float>(ws, L.khat_r));
+            at<float>(ws, L.khat_r), L.kpl_r, L.ksm_r);
     P.total_items = items;
     return from_cuda(launch_pool_project(P, s));
 }
@@ -216,7 +236,7 @@ veda_status do_topk(const veda_problem& p, const Layout& L, int32_t* idx_v, int3
                     cudaStream_t s, uint32_t* status = nullptr)
 {
     if (!idx_v || (L.nr > 0) != (idx_r != nullptr)) return VEDA_ERR_INVALID_ARG;
-    TopkParams T;
+    TopkParams T{};
     T.status = status ? status : at<uint32_t>(ws, 0);
     T.rows = (int64_t)p.B * p.H * L.nq;
     T.scores = at<float>(ws, L.sc_v);
@@ -234,6 +254,60 @@ veda_status do_topk(const veda_problem& p, const Layout& L, int32_t* idx_v, int3
         e = launch_topk(T, s);
     }
     return from_cuda(e);
+}
+
+// Whether veda_select_tiles runs the fused tensor-core score + top-k.
+bool use_fused_selection(const veda_problem& p, const Layout& L)
+{
+    if (p.flags & VEDA_FLAG_UNFUSED_SELECTION) return false;
+    return select_tc_supported(p.r, (int)(L.nq > L.nr ? L.nq : L.nr));
+}
+
+// Steps 2-3 fused: tile scores on the tensor cores and top-k on chip, from the
+// projection planes in the workspace.
+veda_status do_select_fused(const veda_problem& p, const Layout& L, int32_t* idx_v, int32_t* idx_r, void* ws,
+                            cudaStream_t s, uint32_t* status = nullptr)
+{
+    if (!idx_v || (L.nr > 0) != (idx_r != nullptr)) return VEDA_ERR_INVALID_ARG;
+    if (p.r > kPlaneWidth) return VEDA_ERR_UNSUPPORTED;
+    SelectParams S{};
+    S.q_planes = at<uint16_t>(ws, L.qpl);
+    S.BH = p.B * p.H;
+    S.nq = (int32_t)L.nq;
+    S.status = status ? status : at<uint32_t>(ws, 0);
+    S.short_waits = (p.flags & VEDA_FLAG_TEST_SHORT_WAITS) ? 1 : 0;
+    S.n_jobs = L.nr > 0 ? 2 : 1;
+    SelectJob& V = S.job[0];
+    V.k_planes = at<uint16_t>(ws, L.kpl);
+    V.k_sample = at<uint16_t>(ws, L.ksm);
+    V.nk = (int32_t)L.nq;
+    V.k = p.video.budget;
+    V.idx = idx_v;
+    V.sc = at<float>(ws, L.sc_v);
+    V.ld = L.ld_v;
+    V.fb = at<int32_t>(ws, L.fb_v);
+    if (L.nr > 0) {
+        SelectJob& R = S.job[1];
+        R.k_planes = at<uint16_t>(ws, L.kpl_r);
+        R.k_sample = at<uint16_t>(ws, L.ksm_r);
+        R.nk = (int32_t)L.nr;
+        R.k = p.ref.budget;
+        R.idx = idx_r;
+        R.sc = at<float>(ws, L.sc_r);
+        R.ld = L.ld_r;
+        R.fb = at<int32_t>(ws, L.fb_r);
+    }
+    return from_cuda(launch_select_tc(S, s));
+}
+
+// Steps 2-3 on the workspace's projections, fused when supported.
+veda_status do_score_topk(const veda_problem& p, const Layout& L, int32_t* idx_v, int32_t* idx_r, void* ws,
+                          cudaStream_t s, uint32_t* status = nullptr)
+{
+    if (use_fused_selection(p, L)) return do_select_fused(p, L, idx_v, idx_r, ws, s, status);
+    veda_status st = do_score(p, L, ws, s);
+    if (st != VEDA_OK) return st;
+    return do_topk(p, L, idx_v, idx_r, ws, s, status);
 }
 
 veda_status do_attn(const veda_problem& p, const Layout& L, const int32_t* idx_v, const int32_t* idx_r,
@@ -517,8 +591,18 @@ veda_status veda_select_tiles(const veda_problem* p, const void* w_q, const void
     if (!idx_video || (L.nr > 0) != (idx_ref != nullptr)) return VEDA_ERR_INVALID_ARG;
     cudaStream_t s = (cudaStream_t)stream;
     if ((st = do_pool_project(*p, L, w_q, w_k, ws, s)) != VEDA_OK) return st;
-    if ((st = do_score(*p, L, ws, s)) != VEDA_OK) return st;
-    return do_topk(*p, L, idx_video, idx_ref, ws, s);
+    return do_score_topk(*p, L, idx_video, idx_ref, ws, s);
+}
+
+veda_status veda_score_topk_tiles(const veda_problem* p, int32_t* idx_video, int32_t* idx_ref, void* ws,
+                                  size_t ws_bytes, veda_stream_t stream)
+{
+    veda_status st = validate(p);
+    if (st != VEDA_OK) return st;
+    Layout L;
+    if ((st = check_ws(*p, ws, ws_bytes, &L)) != VEDA_OK) return st;
+    if (!idx_video || (L.nr > 0) != (idx_ref != nullptr)) return VEDA_ERR_INVALID_ARG;
+    return do_score_topk(*p, L, idx_video, idx_ref, ws, (cudaStream_t)stream);
 }
 
 veda_status veda_block_sparse_attn(const veda_problem* p, const int32_t* idx_video, const int32_t* idx_ref,
@@ -626,8 +710,7 @@ veda_status veda_attn_host(const veda_problem* p, const void* w_q, const void* w
         if (k_ok) k_ok = cudaStreamWaitEvent(scomp, e_in[sl], 0) == cudaSuccess;
         if (!k_ok) { st = VEDA_ERR_CUDA; break; }
         if ((st = do_pool_project(cp, L, slot + S.wq, slot + S.wk, ws, scomp)) != VEDA_OK) break;
-        if ((st = do_score(cp, L, ws, scomp)) != VEDA_OK) break;
-        if ((st = do_topk(cp, L, iv, ir, ws, scomp, status)) != VEDA_OK) break;
+        if ((st = do_score_topk(cp, L, iv, ir, ws, scomp, status)) != VEDA_OK) break;
         if ((st = do_attn(cp, L, iv, ir, slot + S.out, lse ? reinterpret_cast<float*>(slot + S.lse) : nullptr, ws,
                           scomp, status)) != VEDA_OK)
             break;
@@ -682,8 +765,7 @@ veda_status veda_attn(const veda_problem* p, const void* w_q, const void* w_k, i
     if (!w_q || !w_k || !aligned16(w_q) || !aligned16(w_k)) return VEDA_ERR_INVALID_ARG;
     cudaStream_t s = (cudaStream_t)stream;
     if ((st = do_pool_project(*p, L, w_q, w_k, ws, s)) != VEDA_OK) return st;
-    if ((st = do_score(*p, L, ws, s)) != VEDA_OK) return st;
-    if ((st = do_topk(*p, L, idx_video, idx_ref, ws, s)) != VEDA_OK) return st;
+    if ((st = do_score_topk(*p, L, idx_video, idx_ref, ws, s)) != VEDA_OK) return st;
     return do_attn(*p, L, idx_video, idx_ref, out, lse, ws, s);
 }
 
@@ -695,10 +777,10 @@ veda_status veda_workspace_view(const veda_problem* p, void* ws, size_t ws_bytes
     if (!ptr || !ld) return VEDA_ERR_INVALID_ARG;
     Layout L;
     if ((st = check_ws(*p, ws, ws_bytes, &L)) != VEDA_OK) return st;
-    const size_t offs[5] = {L.qhat, L.khat, L.khat_r, L.sc_v, L.sc_r};
-    const int64_t lds[5] = {p->r, p->r, p->r, L.ld_v, L.ld_r};
-    if (which < 0 || which > 4) return VEDA_ERR_INVALID_ARG;
-    if ((which == 2 || which == 4) && L.nr == 0) return VEDA_ERR_INVALID_ARG;
+    const size_t offs[7] = {L.qhat, L.khat, L.khat_r, L.sc_v, L.sc_r, L.fb_v, L.fb_r};
+    const int64_t lds[7] = {p->r, p->r, p->r, L.ld_v, L.ld_r, 1, 1};
+    if (which < 0 || which > 6) return VEDA_ERR_INVALID_ARG;
+    if ((which == 2 || which == 4 || which == 6) && L.nr == 0) return VEDA_ERR_INVALID_ARG;
     *ptr = static_cast<const char*>(ws) + offs[which];
     *ld = lds[which];
     return VEDA_OK;

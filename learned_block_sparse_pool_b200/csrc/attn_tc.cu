@@ -40,6 +40,7 @@
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
+#include "tc_ptx.cuh"
 #include "veda_internal.cuh"
 
 namespace veda {
@@ -55,7 +56,6 @@ constexpr int kThreads = 320;             // 10 warps: 8 softmax (two groups of 
 // 64 columns), O accumulator of group g at 256 + 128*g.
 __host__ __device__ constexpr uint32_t col_s(uint32_t g) { return 128u * g; }
 __host__ __device__ constexpr uint32_t col_o(uint32_t g) { return 256u + 128u * g; }
-constexpr long long kWaitLimit = 1ll << 31;   // clock cycles (~1 s)
 constexpr float kRescaleThreshold = 8.0f;     // log2 units: rescale O when the max grows > 2^8
 
 struct TcParams {
@@ -118,151 +118,39 @@ struct __align__(1024) Smem {
 };
 
 // ---------------------------------------------------------------- PTX ---
-__device__ __forceinline__ uint32_t smem_u32(const void* p)
+using tc::drain_phase;
+using tc::fence_after;
+using tc::fence_before;
+using tc::idesc_bf16;
+using tc::kWaitLimit;
+using tc::mbar_arrive;
+using tc::mbar_expect_tx;
+using tc::mbar_init;
+using tc::smem_desc;
+using tc::smem_u32;
+using tc::tmem_wait_ld;
+using tc::tmem_wait_st;
+using tc::umma_commit;
+using tc::umma_ss;
+using tc::umma_ts;
+
+__device__ __forceinline__ bool wait_phase(Smem& sm, uint64_t* b, uint32_t parity, uint32_t* status, long long limit)
 {
-    return (uint32_t)__cvta_generic_to_shared(p);
+    return tc::wait_phase(&sm.abort_flag, b, parity, status, limit);
 }
 
-__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count)
+__device__ __forceinline__ bool warp_wait(Smem& sm, uint64_t* b, uint32_t parity, uint32_t* status, long long limit)
 {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* b)
-{
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes)
-{
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* b, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(b)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-__device__ __forceinline__ bool mbar_test_wait(uint64_t* b, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(b)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-constexpr long long kShortWait = 4096;   // limits below this poll without suspending (test hook)
-
-// Bounded wait: true when the phase completed, false on timeout or abort.
-// try_wait may suspend the thread for a while inside one call, so a short
-// (test) limit polls with the non-blocking test_wait instead.
-__device__ __forceinline__ bool wait_phase(Smem& sm, uint64_t* b, uint32_t parity, uint32_t* status,
-                                           long long limit)
-{
-    const bool poll = limit < kShortWait;
-    if (poll ? mbar_test_wait(b, parity) : mbar_try_wait(b, parity)) return true;
-    const long long t0 = clock64();
-    for (;;) {
-        if (poll ? mbar_test_wait(b, parity) : mbar_try_wait(b, parity)) return true;
-        if (sm.abort_flag) return false;
-        if (clock64() - t0 > limit) {
-            record_status(status, VEDA_ERR_TIMEOUT);
-            sm.abort_flag = 1;
-            return false;
-        }
-    }
-}
-
-// Wait by every lane of a warp that next issues warp-collective tcgen05.ld /
-// tcgen05.st: reconverges the warp and makes the outcome warp-uniform.
-__device__ __forceinline__ bool warp_wait(Smem& sm, uint64_t* b, uint32_t parity, uint32_t* status,
-                                          long long limit)
-{
-    const bool ok = wait_phase(sm, b, parity, status, limit);
-    return __all_sync(0xffffffffu, ok);
-}
-
-// Drain wait: like wait_phase but ignores the abort flag (used to let copies
-// and MMAs already in flight land before the CTA releases its resources).
-__device__ __forceinline__ bool drain_phase(uint64_t* b, uint32_t parity, uint32_t* status)
-{
-    const long long t0 = clock64();
-    while (!mbar_try_wait(b, parity)) {
-        if (clock64() - t0 > kWaitLimit) {
-            record_status(status, VEDA_ERR_TIMEOUT);
-            return false;
-        }
-    }
-    return true;
+    return tc::warp_wait(&sm.abort_flag, b, parity, status, limit);
 }
 
 __device__ __forceinline__ void tma_load(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1, int c2,
                                          int c3)
 {
-    asm volatile(
-        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], "
-        "[%6];" ::"r"(smem_u32(dst)),
-        "l"((uint64_t)map), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
-        : "memory");
+    tc::tma_load_4d(dst, map, bar, c0, c1, c2, c3);
 }
 
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-// The MMA helpers below are executed by all 32 lanes of the issuing warp
-// with warp-uniform operands; one lane, chosen by elect.sync, issues.
-__device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                        uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p, e;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                        uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p, e;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-__device__ __forceinline__ void umma_commit(uint64_t* bar)
-{
-    asm volatile(
-        "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
-        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar))
-        : "memory");
-}
-
-#define TMEM_LD32(taddr, r)                                                                                      \
-    asm volatile(                                                                                                \
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17," \
-        "%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"                                       \
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),        \
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),  \
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]),             \
-          "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),             \
-          "=r"(r[30]), "=r"(r[31])                                                                               \
-        : "r"(taddr))
+#define TMEM_LD32(taddr, r) VEDA_TMEM_LD32(taddr, r)
 
 #define TMEM_ST32(taddr, r)                                                                                      \
     asm volatile(                                                                                                \
@@ -281,8 +169,6 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar)
         "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])            \
         : "memory")
 
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ float fast_exp2(float x)
 {
@@ -323,20 +209,6 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b)
     uint64_t d;
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
-}
-
-// Shared-memory matrix descriptor, 128-byte swizzle, sm100 format (version 1).
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo)
-{
-    return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
-}
-
-// Instruction descriptor: bf16 x bf16 -> fp32, M = 128, N = 128.
-__host__ __device__ constexpr uint32_t idesc_bf16(bool b_mn_major)
-{
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(128 >> 3) << 17) |
-           ((uint32_t)(128 >> 4) << 24);
 }
 
 // ------------------------------------------------------------ tile list ---
@@ -411,9 +283,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    tc_fence_before();
+    fence_before();
     __syncthreads();
-    tc_fence_after();
+    fence_after();
     const uint32_t tmem = sm.tmem_base;
 
     if (warp == kProducerWarp && lane == 0) {
@@ -469,12 +341,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             const int nl = kSplit ? unit_ref<kSplit>(P, u, n_list).nl : n_list;
             if (!(ok = warp_wait(sm, &sm.q_full, uq & 1, P.status, P.wait_limit))) break;
             ++uq;
-            tc_fence_after();
+            fence_after();
             const uint32_t qaddr = smem_u32(sm.q);
             auto issue_s = [&](int j) -> bool {
                 const uint32_t st = kst, g = j & 1;
                 if (!warp_wait(sm, &sm.kv_full[st], kph, P.status, P.wait_limit)) return false;
-                tc_fence_after();
+                fence_after();
                 const uint32_t kaddr = smem_u32(sm.kv[st]);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
@@ -497,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 if (j == 0 && units_done > 0 &&
                     !(ok = warp_wait(sm, &sm.o_free, (units_done - 1) & 1, P.status, P.wait_limit)))
                     break;
-                tc_fence_after();
+                fence_after();
                 const uint32_t vaddr = smem_u32(sm.kv[st]);
 #pragma unroll
                 for (int kk = 0; kk < TT / 16; ++kk)
@@ -538,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 const TileRef r = r_next;
                 if (j + 2 < nl) r_next = resolve(P, urow, j0 + j + 2);   // one tile ahead
                 if (!(ok = warp_wait(sm, &sm.s_full[g], sc & 1, P.status, P.wait_limit))) break;
-                tc_fence_after();
+                fence_after();
                 uint32_t s[128];
                 const uint32_t sa = tmem + lane_off + col_s(g);
                 TMEM_LD32(sa + 0, (s + 0));
@@ -609,7 +481,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 // rewrites its 32 rows of O (factor 1 where the max is kept).
                 if (__any_sync(0xffffffffu, rescale)) {
                     if (!(ok = warp_wait(sm, &sm.pv_done[g], (sc - 1) & 1, P.status, P.wait_limit))) break;
-                    tc_fence_after();
+                    fence_after();
                     const float a = rescale ? alpha : 1.f;
                     const uint32_t oa = tmem + lane_off + col_o(g);
 #pragma unroll
@@ -623,7 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                     }
                     tmem_wait_st();
                 }
-                tc_fence_before();
+                fence_before();
                 mbar_arrive(&sm.p_full[g]);
             }
             if (!ok) break;
@@ -635,7 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             sm.red_l[up][g][row] = l;
             mbar_arrive(&sm.xchg[wq]);
             if (!(ok = warp_wait(sm, &sm.xchg[wq], uu & 1, P.status, P.wait_limit))) break;
-            tc_fence_after();
+            fence_after();
             const float m0 = sm.red_m[up][0][row], m1 = sm.red_m[up][1][row];
             const float l0 = sm.red_l[up][0][row], l1 = sm.red_l[up][1][row];
             const float M = fmaxf(m0, m1);
@@ -698,15 +570,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             } else if (P.lse && g == 0 && tok < P.n_qtok) {
                 P.lse[((int64_t)b * P.H + h) * P.n_qtok + tok] = (M + __log2f(L)) * 0.69314718055994531f;
             }
-            tc_fence_before();
+            fence_before();
             mbar_arrive(&sm.o_free);
         }
     }
 
     // ---------------------------------------------------- teardown ---
-    tc_fence_before();
+    fence_before();
     __syncthreads();
-    tc_fence_after();
+    fence_after();
     if (warp == kMmaWarp) {
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512) : "memory");
     }
@@ -752,15 +624,7 @@ __global__ void __launch_bounds__(256) merge_splits_kernel(const float* __restri
 }
 
 // ------------------------------------------------------------------ host ---
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
-{
-    void* fn = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-        return nullptr;
-    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-}
+using tc::encode_fn;
 
 // Tensor map over a [B, n, H, 128] bf16 tensor (element strides sb, st, sh),
 // box = 64 channels x 128 tokens of one (b, h); dims 1..3 ordered by stride.

@@ -27,6 +27,7 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kMaxTile = 128;
+constexpr int kPlaneWidth = 64;   // columns of a bf16 plane row (r <= 64, zero padded)
 
 __device__ __forceinline__ void unpack(const uint4& raw, float* f, const float*)
 {
@@ -167,13 +168,39 @@ __global__ void __launch_bounds__(kThreads) pool_project_kernel(const PoolParams
         // projection of the round's pooled vectors: one output (g, c) per thread
         const int hh = cur_h;
         const int bb = (int)(((it - ng - J.first_item) / J.n_tiles) / P.H);
-        for (int x = tid; x < ng * r; x += kThreads) {
-            const int g = x / r, c = x % r;
-            const float* pv = pooled + g * D;
+        const int rc = J.planes ? kPlaneWidth : r;   // columns written per tile
+        for (int x = tid; x < ng * rc; x += kThreads) {
+            const int g = x / rc, c = x % rc;
+            const int64_t orow = (int64_t)(bb * P.H + hh) * J.n_tiles + i0 + g;
             float s = 0.f;
+            if (c < r) {
+                const float* pv = pooled + g * D;
 #pragma unroll 8
-            for (int e = 0; e < D; ++e) s = fmaf(pv[e], w_s[e * r + c], s);
-            J.out[((int64_t)(bb * P.H + hh) * J.n_tiles + i0 + g) * r + c] = s;
+                for (int e = 0; e < D; ++e) s = fmaf(pv[e], w_s[e * r + c], s);
+                J.out[orow * r + c] = s;
+            }
+            if (J.planes) {
+                // three bf16 terms summing to s: each difference is exact in fp32
+                const __nv_bfloat16 p0 = __float2bfloat16_rn(s);
+                const float r1 = s - __bfloat162float(p0);
+                const __nv_bfloat16 p1 = __float2bfloat16_rn(r1);
+                const __nv_bfloat16 p2 = __float2bfloat16_rn(r1 - __bfloat162float(p1));
+                uint16_t* dst = J.planes + orow * kPlaneWidth + c;
+                dst[0] = __bfloat16_as_ushort(p0);
+                dst[J.plane_stride] = __bfloat16_as_ushort(p1);
+                dst[2 * J.plane_stride] = __bfloat16_as_ushort(p2);
+                if (J.sample_planes) {
+                    // sample rows m with floor(m n / 64) == this tile: 64 i <= m n < 64 (i + 1)
+                    const int64_t n = J.n_tiles, ti = i0 + g;
+                    const int64_t m_lo = (64 * ti + n - 1) / n, m_hi = min((int64_t)63, (64 * (ti + 1) + n - 1) / n - 1);
+                    for (int64_t m = m_lo; m <= m_hi; ++m) {
+                        uint16_t* sd = J.sample_planes + ((int64_t)(bb * P.H + hh) * 64 + m) * kPlaneWidth + c;
+                        sd[0] = __bfloat16_as_ushort(p0);
+                        sd[J.sample_plane_stride] = __bfloat16_as_ushort(p1);
+                        sd[2 * J.sample_plane_stride] = __bfloat16_as_ushort(p2);
+                    }
+                }
+            }
         }
     }
 }

@@ -239,8 +239,9 @@ __global__ void __launch_bounds__(32 * kWarps, 4) topk_kernel(const TopkParams P
     const uint32_t lt_mask = (1u << lane) - 1u;
     const bool sampled = n > kSample && r_lo < kSample - 1;
 
-    for (int64_t row = (int64_t)blockIdx.x * kWarps + w; row < P.rows;
-         row += (int64_t)gridDim.x * kWarps) {
+    const int64_t n_rows = P.row_list ? (int64_t)*P.row_count : P.rows;
+    for (int64_t rr = (int64_t)blockIdx.x * kWarps + w; rr < n_rows; rr += (int64_t)gridDim.x * kWarps) {
+        const int64_t row = P.row_list ? (int64_t)P.row_list[rr] : rr;
         const float* src = P.scores + row * P.ld;
         int32_t* dst = P.idx + row * (int64_t)k;
 
@@ -437,9 +438,10 @@ cudaError_t launch_topk(const TopkParams& p, cudaStream_t s)
     if (e != cudaSuccess) return e;
     if (per_sm < 1) per_sm = 1;
     int64_t grid = (int64_t)num_sms() * per_sm;
-    const int64_t need = (p.rows + kWarps - 1) / kWarps;
+    const int64_t need = (p.rows + kWarps - 1) / kWarps;   // a row list is never longer than `rows`
     if (grid > need) grid = need;
-        const int r_lo = p.n > kSample ? bracket_rank(p.n, p.k) : kSample - 1;
+    if (p.row_list && !p.row_count) return cudaErrorInvalidValue;
+    const int r_lo = p.n > kSample ? bracket_rank(p.n, p.k) : kSample - 1;
     topk_kernel<<<(unsigned)grid, 32 * kWarps, smem, s>>>(p, cap, r_lo);
     return cudaGetLastError();
 }

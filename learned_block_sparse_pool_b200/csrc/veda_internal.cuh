@@ -34,6 +34,16 @@ struct PoolJob {
     float* out;             // [B, H, n_tiles, r]
     int32_t n_tiles;
     int32_t pad;
+    // optional (nullptr: none): the projections again as three bf16 planes
+    // [3][B H][n_tiles][64] whose sum is the fp32 value (x = p0 + p1 + p2,
+    // p0 = bf16(x), p1 = bf16(x - p0), p2 = bf16(x - p0 - p1)), columns
+    // r..63 zero: the operands of the tensor-core tile scoring
+    uint16_t* planes;
+    int64_t plane_stride;   // elements from one plane to the next
+    // optional (nullptr: none): the planes of the kSample tiles the fused
+    // selection samples, [3][B H][64][64]: sample m is tile (m n_tiles) / 64
+    uint16_t* sample_planes;
+    int64_t sample_plane_stride;
 };
 
 struct PoolParams {
@@ -57,6 +67,36 @@ struct ScoreParams {
 
 cudaError_t launch_score(const ScoreParams& p, cudaStream_t s);
 
+// ---- fused tile scoring + top-k on the tensor cores -----------------------
+// Scores s[i][j] = qhat_i . khat_j are computed on the tensor cores from the
+// bf16 planes written by the pool + project kernel (six plane products: fp32
+// accuracy) and never stored; every row's top-k is selected on chip (see
+// select_rows.cuh).  Rows whose selection needs the exact fallback get their
+// scores written to `sc` and their row id appended to `fb` (fb[0] = count);
+// launch_topk_rows then finishes them.
+struct SelectJob {
+    const uint16_t* k_planes;   // [3][BH][nk][64]
+    const uint16_t* k_sample;   // [3][BH][64][64]: the planes of the sampled tiles
+    int32_t nk;                 // key tiles
+    int32_t k;                  // budget
+    int32_t* idx;               // [BH][nq][k]
+    float* sc;                  // [BH][nq][ld] fallback scores
+    int64_t ld;
+    int32_t* fb;                // [1 + BH nq]
+};
+
+struct SelectParams {
+    const uint16_t* q_planes;   // [3][BH][nq][64]
+    SelectJob job[2];
+    int32_t n_jobs;
+    int32_t BH, nq;
+    uint32_t* status;
+    int32_t short_waits;
+};
+
+bool select_tc_supported(int r, int n_tiles_max);
+cudaError_t launch_select_tc(const SelectParams& p, cudaStream_t s);
+
 // ---- fixed-budget top-k -------------------------------------------------
 struct TopkParams {
     const float* scores;    // [rows, ld]
@@ -66,9 +106,13 @@ struct TopkParams {
     int32_t k;              // budget
     int32_t* idx;           // [rows, k]
     uint32_t* status;
+    // optional: process only the rows listed in row_list[0 .. *row_count)
+    const int32_t* row_list;
+    const int32_t* row_count;
 };
 
 cudaError_t launch_topk(const TopkParams& p, cudaStream_t s);
+int topk_max_tiles();
 
 // ---- attention ----------------------------------------------------------
 struct AttnParams {

@@ -97,9 +97,14 @@ def test_valid_problem_workspace_size(L):
     nq, nr = 8, 3
     ld_v, ld_r = 32, 32
     BH, r = 4, 64
-    # status block + qhat + khat + khat_ref + scores + scores_ref, each 256-aligned
+    # status block + qhat + khat + khat_ref + scores + scores_ref + the three
+    # bf16 projection planes (q, k, k_ref: 3 x 64 columns) and of the 64
+    # sampled key tiles (video, reference) + the two lists of
+    # rows left to the exact top-k by the fused selection, each 256-aligned
     expect = 256
-    for nbytes in (4 * BH * nq * r, 4 * BH * nq * r, 4 * BH * nr * r, 4 * BH * nq * ld_v, 4 * BH * nq * ld_r):
+    for nbytes in (4 * BH * nq * r, 4 * BH * nq * r, 4 * BH * nr * r, 4 * BH * nq * ld_v, 4 * BH * nq * ld_r,
+                   6 * BH * nq * 64, 6 * BH * nq * 64, 6 * BH * nr * 64, 6 * BH * 64 * 64, 6 * BH * 64 * 64,
+                   4 * (1 + BH * nq), 4 * (1 + BH * nq)):
         expect += -(-nbytes // 256) * 256
     assert n == expect
 
@@ -111,7 +116,7 @@ def test_valid_problem_workspace_size(L):
     ({"r": 132}, B.VEDA_ERR_UNSUPPORTED),
     ({"B": 0}, B.VEDA_ERR_INVALID_ARG),
     ({"dtype": 7}, B.VEDA_ERR_INVALID_ARG),
-    ({"flags": 4}, B.VEDA_ERR_INVALID_ARG),
+    ({"flags": 8}, B.VEDA_ERR_INVALID_ARG),
     ({"softmax_scale": -1.0}, B.VEDA_ERR_INVALID_ARG),
     ({"softmax_scale": float("nan")}, B.VEDA_ERR_INVALID_ARG),
     ({"q": 0}, B.VEDA_ERR_INVALID_ARG),
@@ -135,7 +140,7 @@ def test_invalid_arguments_rejected_on_host(L, over, code):
 
 
 def test_test_hook_flags_are_accepted(L):
-    for flags in (B.VEDA_FLAG_SIMT_ATTENTION, B.VEDA_FLAG_TEST_SHORT_WAITS, 3):
+    for flags in (B.VEDA_FLAG_SIMT_ATTENTION, B.VEDA_FLAG_TEST_SHORT_WAITS, B.VEDA_FLAG_UNFUSED_SELECTION, 7):
         st, _ = _ws_size(L, _problem(flags=flags))
         assert st == B.VEDA_OK
 
@@ -240,7 +245,11 @@ def test_workspace_view_bounds(L):
     assert ptr.value == 0x800000 + 256 and ld.value == 64
     assert L.veda_workspace_view(ctypes.byref(p), 0x800000, n, 2, ctypes.byref(ptr), ctypes.byref(ld)) == \
         B.VEDA_ERR_INVALID_ARG
-    assert L.veda_workspace_view(ctypes.byref(p), 0x800000, n, 5, ctypes.byref(ptr), ctypes.byref(ld)) == \
+    assert L.veda_workspace_view(ctypes.byref(p), 0x800000, n, 5, ctypes.byref(ptr), ctypes.byref(ld)) == B.VEDA_OK
+    assert ld.value == 1 and 0x800000 < ptr.value < 0x800000 + n
+    assert L.veda_workspace_view(ctypes.byref(p), 0x800000, n, 6, ctypes.byref(ptr), ctypes.byref(ld)) == \
+        B.VEDA_ERR_INVALID_ARG
+    assert L.veda_workspace_view(ctypes.byref(p), 0x800000, n, 7, ctypes.byref(ptr), ctypes.byref(ld)) == \
         B.VEDA_ERR_INVALID_ARG
 
 

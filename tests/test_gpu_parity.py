@@ -348,6 +348,9 @@ def test_full_size_workload(dev, oracle_mod, name):
     sel = oracle_mod.select_tiles(host, w.T, w.budget_video, w.budget_ref if w.ref_frames else 0)
     rep = check_selection(oracle_mod, p, ws, iv, ir, sel, name, host)
     _report(name, rep)
+    fb = len(veda.fallback_rows(p, ws))
+    warnings.warn(f"{name}: {fb} of {rep.rows} rows finished by the exact step-3 kernel", TieBandReport)
+    assert fb <= rep.rows // 100
     units = sample_units(w, n_units=64 if name in FULL else 24)
     _, err = check_attention(oracle_mod, w, host, p, ws, sel, units, name)
     print(f"{name}: attention on {len(units)} units: max-abs {err[0]:.3g} rel-L2 {err[1]:.3g}")

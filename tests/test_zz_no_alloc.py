@@ -5,7 +5,8 @@ take cudaMalloc's device synchronisation).  Its scratch is a static per-device
 array inside the library, so the caller passes only inputs and outputs.
 
 Checked through the C ABI against veda_select_tiles (the workspace entry
-point): the kept tiles must be identical, on two calls in a row (the static
+point) running the same kernels (VEDA_FLAG_UNFUSED_SELECTION): the kept tiles
+must be identical, on two calls in a row (the static
 array keeps the previous call's contents, which must not leak into the next
 result).  pytest collects this file last (its name sorts last), so a run that
 stops at the first failure has run every other test before this one; the
@@ -30,15 +31,17 @@ def dev():
     return torch.device("cuda:0")
 
 
-def _problem(w, g):
+def _problem(w, g, flags=0):
     return veda.Problem(g["q"], g["k"], g["v"], tile=w.T, r=w.r, budget=w.budget_video,
                         k_ref=g.get("k_ref"), v_ref=g.get("v_ref"),
                         budget_ref=w.budget_ref if "k_ref" in g else 0,
-                        k_dense=g.get("k_dense"), v_dense=g.get("v_dense"))
+                        k_dense=g.get("k_dense"), v_dense=g.get("v_dense"), flags=flags)
 
 
 def _compare_two_calls(w, g):
-    p = _problem(w, g)
+    # the workspace entry point on the same kernels (fp32 SIMT scores, then
+    # the warp-per-row top-k), so the kept tiles must be identical
+    p = _problem(w, g, flags=B.VEDA_FLAG_UNFUSED_SELECTION)
     ws = veda.workspace(p)
     iv, ir = veda.alloc_indices(p)
     veda.select_tiles(p, g["w_q"], g["w_k"], iv, ir, ws)
