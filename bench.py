@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--simt", action="store_true", help="use the SIMT attention kernel")
     ap.add_argument("--unfused-selection", action="store_true",
                     help="time the three-kernel selection (fp32 SIMT scores, then the warp-per-row top-k)")
+    ap.add_argument("--onchip-selection", action="store_true",
+                    help="time the on-chip selection (tensor-core scores recomputed per pass, no score matrix)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ncu", action="store_true", help="short run for profiler captures (no extras)")
@@ -213,12 +215,12 @@ def bench_config(w, n, simt=False):
     })
 
 
-def make_problem(veda, w, g, simt=False):
+def make_problem(veda, w, g, simt=False, flags=0):
     return veda.Problem(g["q"], g["k"], g["v"], tile=w.T, r=w.r, budget=w.budget_video,
                         k_ref=g.get("k_ref"), v_ref=g.get("v_ref"),
                         budget_ref=w.budget_ref if "k_ref" in g else 0,
                         k_dense=g.get("k_dense"), v_dense=g.get("v_dense"),
-                        flags=veda.binding.VEDA_FLAG_SIMT_ATTENTION if simt else 0)
+                        flags=(veda.binding.VEDA_FLAG_SIMT_ATTENTION if simt else 0) | flags)
 
 
 def main():
@@ -255,7 +257,9 @@ def main():
 
     import learned_block_sparse_pool_b200 as veda
     g = workloads.make_inputs(w, device=dev)
-    p = make_problem(veda, w, g, args.simt)
+    sel_flags = (veda.binding.VEDA_FLAG_UNFUSED_SELECTION if args.unfused_selection else 0) | \
+        (veda.binding.VEDA_FLAG_ONCHIP_SELECTION if args.onchip_selection else 0)
+    p = make_problem(veda, w, g, args.simt, sel_flags)
     ws = veda.workspace(p)
     if args.dense_queries:
         dense_query_run(args, veda, w, g, p, ws, dev, local, rank, n, dist)
@@ -350,18 +354,30 @@ def main():
             "score_gflops": round(score_flop / (st_ms["score"] / 1e3) / 1e9, 1),
         })
         launches_per_step = 2 + 2 * len(segs)
-    else:
-        # fused score + top-k: reads the bf16 projection planes (k-hat from L2)
-        # and writes the kept indices; its work is the tensor-core scoring of
-        # every (query tile, key tile) pair, repeated for each pass
+    elif args.onchip_selection:
+        # one kernel: tensor-core scores recomputed per pass, top-k on chip;
+        # reads the bf16 projection planes (k-hat from L2) and writes the kept indices
         sel_bytes = sum(rows * k * 4 for _, k in segs) + 6 * 64 * rows * (1 + len(segs))
         selector.update({
-            "select_kernel": "fused tensor-core score + on-chip top-k (no score matrix in HBM)",
+            "select_kernel": "tensor-core scores + on-chip top-k (no score matrix in HBM)",
             "select_ms": round(st_ms["select"], 4),
             "select_algorithmic_bytes": sel_bytes,
             "select_score_gflops": round(score_flop / (st_ms["select"] / 1e3) / 1e9, 1),
         })
-        launches_per_step = 3 + sum(1 for nk, k in segs if 128 < nk and k < nk)   # + fallback top-k
+        launches_per_step = 3 + sum(1 for nk, k in segs if k < nk)   # + the top-k of rows left over
+    else:
+        # tensor-core scores written once (exact), then the warp-per-row top-k
+        # reads them: planes in, scores out and back in, indices out
+        sel_bytes = sum(rows * (2 * nk * 4 + k * 4) for nk, k in segs) + 6 * 64 * rows * (1 + len(segs))
+        selector.update({
+            "select_kernels": "tensor-core scores to HBM + warp-per-row top-k",
+            "select_ms": round(st_ms["select"], 4),
+            "select_algorithmic_bytes": sel_bytes,
+            "select_gbs": round(sel_bytes / (st_ms["select"] / 1e3) / 1e9, 1),
+            "select_frac": round(sel_bytes / (st_ms["select"] / 1e3) / 1e9 / hbm, 4),
+            "select_score_gflops": round(score_flop / (st_ms["select"] / 1e3) / 1e9, 1),
+        })
+        launches_per_step = 3 + len(segs)
 
     res = {
         "metric": METRIC,

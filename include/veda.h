@@ -90,13 +90,17 @@ typedef enum { VEDA_F32 = 0, VEDA_BF16 = 1 } veda_dtype;
                                        reports VEDA_ERR_TIMEOUT through
                                        veda_check_status(); its output is then
                                        undefined.  No effect on other kernels. */
-#define VEDA_FLAG_UNFUSED_SELECTION 4u /* select tiles with the three-kernel path
-                                       (fp32 SIMT scores written to the
-                                       workspace, then the warp-per-row top-k)
-                                       instead of the fused tensor-core score +
-                                       top-k: a cross-check path.  The fused
-                                       path needs r <= 64 and falls back to
-                                       this one otherwise. */
+#define VEDA_FLAG_UNFUSED_SELECTION 4u /* compute the tile scores with the fp32
+                                       SIMT kernel instead of the tensor cores
+                                       (a cross-check path; also used when
+                                       r > 64) */
+#define VEDA_FLAG_ONCHIP_SELECTION 8u /* select each row's top-k on chip while
+                                       the tensor cores recompute its scores,
+                                       writing no score matrix (see
+                                       veda_score_topk_tiles); otherwise the
+                                       tensor-core scores are written to the
+                                       workspace and the warp-per-row top-k
+                                       kernel selects from them */
 
 /* One key/value segment, [B, n_tokens, H, d] (d contiguous). */
 typedef struct {
@@ -141,9 +145,8 @@ VEDA_API veda_status veda_workspace_init(void* ws, size_t ws_bytes, veda_stream_
 
 /* Steps 1-3: pool + project Q and K, score every key tile, keep the top
  * `budget` per (b, h, query tile) for the video segment and, when present,
- * independently for the reference segment.  Steps 2-3 run fused on the
- * tensor cores (see veda_score_topk_tiles) unless r > 64 or
- * VEDA_FLAG_UNFUSED_SELECTION is set.
+ * independently for the reference segment.  Steps 2-3 run as
+ * veda_score_topk_tiles describes.
  *   w_q, w_k   [H, d, r] device, problem dtype
  *   idx_video  [B, H, n_q_tiles, video.budget] int32 out (ascending rows)
  *   idx_ref    [B, H, n_q_tiles, ref.budget]   int32 out; NULL iff no reference */
@@ -231,14 +234,17 @@ VEDA_API veda_status veda_score_tiles(const veda_problem* p, void* ws, size_t ws
 /* Step 3: top-k of the workspace scores into idx_video / idx_ref. */
 VEDA_API veda_status veda_topk_tiles(const veda_problem* p, int32_t* idx_video, int32_t* idx_ref,
                             void* ws, size_t ws_bytes, veda_stream_t stream);
-/* Steps 2-3 fused (what veda_select_tiles runs after veda_pool_project): the
+/* Steps 2-3 (what veda_select_tiles runs after veda_pool_project).  The
  * tile scores are computed on the tensor cores from the projections in the
  * workspace, as three bf16 parts per value whose six leading products give
- * fp32 accuracy, and each row's top-k is selected on chip without writing
- * the score matrix; rows whose on-chip selection cannot finish (a score band
- * wider than its buffer, or a NaN) get their scores written to the
- * workspace and go through the step-3 kernel.  With r > 64 or
- * VEDA_FLAG_UNFUSED_SELECTION this runs steps 2 and 3 unfused. */
+ * fp32 accuracy.  By default they are written to the workspace and the
+ * step-3 kernel selects from them.  With VEDA_FLAG_ONCHIP_SELECTION the same
+ * kernel selects each row's top-k on chip while it recomputes the row's
+ * scores pass by pass, writing no score matrix; rows whose on-chip
+ * selection cannot finish (a score band wider than its buffer, or a NaN) get
+ * their scores written to the workspace and go through the step-3 kernel.
+ * With r > 64 or VEDA_FLAG_UNFUSED_SELECTION the scores come from the fp32
+ * SIMT kernel. */
 VEDA_API veda_status veda_score_topk_tiles(const veda_problem* p, int32_t* idx_video, int32_t* idx_ref,
                                            void* ws, size_t ws_bytes, veda_stream_t stream);
 

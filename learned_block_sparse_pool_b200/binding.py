@@ -29,6 +29,7 @@ VEDA_F32, VEDA_BF16 = 0, 1
 VEDA_FLAG_SIMT_ATTENTION = 1
 VEDA_FLAG_TEST_SHORT_WAITS = 2
 VEDA_FLAG_UNFUSED_SELECTION = 4
+VEDA_FLAG_ONCHIP_SELECTION = 8
 
 EXPORTS = ("veda_workspace_size", "veda_workspace_init", "veda_select_tiles", "veda_block_sparse_attn",
            "veda_attn", "veda_pool_project", "veda_score_tiles", "veda_topk_tiles", "veda_workspace_view",
@@ -279,7 +280,8 @@ def topk_tiles(p: Problem, idx_v, idx_r, ws, stream=None) -> None:
 
 
 def score_topk_tiles(p: Problem, idx_v, idx_r, ws, stream=None) -> None:
-    """Steps 2-3 (fused on the tensor cores unless unsupported or flagged)."""
+    """Steps 2-3: tensor-core scores, then the top-k (on chip with
+    VEDA_FLAG_ONCHIP_SELECTION; SIMT scores with VEDA_FLAG_UNFUSED_SELECTION)."""
     _check(lib().veda_score_topk_tiles(p.ref(), _ptr(idx_v), _ptr(idx_r), ws.data_ptr(), ws.numel(),
                                        _stream(stream)), "veda_score_topk_tiles")
 

@@ -113,7 +113,8 @@ veda_status validate(const veda_problem* pp)
     if (p.tile != 64 && p.tile != 128) return VEDA_ERR_UNSUPPORTED;
     if (p.r > 128 || p.r % 4 != 0) return VEDA_ERR_UNSUPPORTED;
     if (!(p.softmax_scale >= 0.f) || !isfinite(p.softmax_scale)) return VEDA_ERR_INVALID_ARG;
-    if (p.flags & ~(VEDA_FLAG_SIMT_ATTENTION | VEDA_FLAG_TEST_SHORT_WAITS | VEDA_FLAG_UNFUSED_SELECTION))
+    if (p.flags & ~(VEDA_FLAG_SIMT_ATTENTION | VEDA_FLAG_TEST_SHORT_WAITS | VEDA_FLAG_UNFUSED_SELECTION |
+                    VEDA_FLAG_ONCHIP_SELECTION))
         return VEDA_ERR_INVALID_ARG;
     if (!p.q || !aligned16(p.q)) return VEDA_ERR_INVALID_ARG;
     const size_t es = esize(p.dtype);
@@ -256,21 +257,25 @@ veda_status do_topk(const veda_problem& p, const Layout& L, int32_t* idx_v, int3
     return from_cuda(e);
 }
 
-// Whether veda_select_tiles runs the fused tensor-core score + top-k.
-bool use_fused_selection(const veda_problem& p, const Layout& L)
+// Whether the tile scores are computed on the tensor cores (from the bf16
+// projection planes) rather than by the fp32 SIMT kernel.
+bool use_tensor_scores(const veda_problem& p, const Layout& L)
 {
     if (p.flags & VEDA_FLAG_UNFUSED_SELECTION) return false;
     return select_tc_supported(p.r, (int)(L.nq > L.nr ? L.nq : L.nr));
 }
 
-// Steps 2-3 fused: tile scores on the tensor cores and top-k on chip, from the
-// projection planes in the workspace.
-veda_status do_select_fused(const veda_problem& p, const Layout& L, int32_t* idx_v, int32_t* idx_r, void* ws,
-                            cudaStream_t s, uint32_t* status = nullptr)
+// Steps 2-3 on the tensor cores, from the projection planes in the
+// workspace: with scores_only the exact scores are written to the
+// workspace (then the warp-per-row top-k runs); otherwise each row's top-k
+// is selected on chip and no score matrix is written.
+veda_status do_select_tc(const veda_problem& p, const Layout& L, int32_t* idx_v, int32_t* idx_r, void* ws,
+                         cudaStream_t s, uint32_t* status, bool scores_only)
 {
     if (!idx_v || (L.nr > 0) != (idx_r != nullptr)) return VEDA_ERR_INVALID_ARG;
     if (p.r > kPlaneWidth) return VEDA_ERR_UNSUPPORTED;
     SelectParams S{};
+    S.scores_only = scores_only ? 1 : 0;
     S.q_planes = at<uint16_t>(ws, L.qpl);
     S.BH = p.B * p.H;
     S.nq = (int32_t)L.nq;
@@ -300,12 +305,20 @@ veda_status do_select_fused(const veda_problem& p, const Layout& L, int32_t* idx
     return from_cuda(launch_select_tc(S, s));
 }
 
-// Steps 2-3 on the workspace's projections, fused when supported.
+// Steps 2-3 on the workspace's projections: tensor-core scores and the
+// warp-per-row top-k by default, the on-chip selection with
+// VEDA_FLAG_ONCHIP_SELECTION, fp32 SIMT scores with VEDA_FLAG_UNFUSED_SELECTION
+// (or when the tensor-core path does not apply).
 veda_status do_score_topk(const veda_problem& p, const Layout& L, int32_t* idx_v, int32_t* idx_r, void* ws,
                           cudaStream_t s, uint32_t* status = nullptr)
 {
-    if (use_fused_selection(p, L)) return do_select_fused(p, L, idx_v, idx_r, ws, s, status);
-    veda_status st = do_score(p, L, ws, s);
+    veda_status st;
+    if (use_tensor_scores(p, L)) {
+        if (p.flags & VEDA_FLAG_ONCHIP_SELECTION) return do_select_tc(p, L, idx_v, idx_r, ws, s, status, false);
+        st = do_select_tc(p, L, idx_v, idx_r, ws, s, status, true);
+    } else {
+        st = do_score(p, L, ws, s);
+    }
     if (st != VEDA_OK) return st;
     return do_topk(p, L, idx_v, idx_r, ws, s, status);
 }

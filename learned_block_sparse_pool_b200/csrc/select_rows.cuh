@@ -216,8 +216,8 @@ VEDA_HD void finish_count(Row& R, const int (&c)[kM], int k)
 // where the k-th score would lie if the band's scores were spread evenly (the
 // (k - above)-th of `band` from the top), at offsets of 4 % to 55 % of the
 // band's width on either side (finer where the k-th score is expected), and
-// reaching 5 % of the width past both ends, so that pass A's counts (which
-// may come from approximate scores) are not needed to place the k-th score.
+// reaching past both ends, so that pass A's counts (which may come from
+// approximate scores) are not needed to place the k-th score.
 // The band is then re-derived from pass B's counts alone (restart_ladder).
 VEDA_HD void plan_in_band(Row& R, int k)
 {
@@ -227,8 +227,12 @@ VEDA_HD void plan_in_band(Row& R, int k)
     const float f = ((float)(k - R.above) - 0.5f) / (float)(R.band > 0 ? R.band : 1);
     const float xc = hi - f * w;
     const float off[kM] = {0.55f, 0.3f, 0.12f, 0.04f, -0.04f, -0.12f, -0.3f, -0.55f};
+    // past the ends: 5 % of the width, and at least 16 g units (about 1 % of
+    // the sampled bracket), which covers the error of pass A's approximate
+    // scores when the band is very narrow (a budget of one or two tiles)
+    const float mg = 0.05f * w + 16.0f;
 #pragma unroll
-    for (int i = 0; i < kM; ++i) R.t[i] = f16_round(fminf(fmaxf(xc + off[i] * w, lo - 0.05f * w), hi + 0.05f * w));
+    for (int i = 0; i < kM; ++i) R.t[i] = f16_round(fminf(fmaxf(xc + off[i] * w, lo - mg), hi + mg));
 #pragma unroll
     for (int i = 1; i < kM; ++i) R.t[i] = fminf(R.t[i], R.t[i - 1]);   // non-increasing after rounding
 }

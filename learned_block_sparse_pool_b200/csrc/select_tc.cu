@@ -65,10 +65,10 @@ constexpr uint32_t kColS = 128;                 // score buffers: kNB x 64 colum
 static_assert(rs::kSample == kCols && rs::kCap == kCols, "the sample and band sorts share one 64-value network");
 
 // Passes of a unit: the sample chunk, then nc chunks per pass.
-enum { kSamplePass = 0, kCountA = 1, kCountB = 2, kCollect = 3, kEmit = 4 };
+enum { kSamplePass = 0, kCountA = 1, kCountB = 2, kCollect = 3, kEmit = 4, kStore = 5 };
 
 struct JobDev {
-    int32_t nk, k, nc, mode;   // mode 0: every tile kept; 2: selected on chip
+    int32_t nk, k, nc, mode;   // mode 0: every tile kept; 2: selected on chip; 3: scores written out
     int32_t* idx;
     float* sc;
     int64_t ld;
@@ -98,9 +98,15 @@ struct __align__(1024) Smem {
     volatile int abort_flag;
 };
 
+// Chunks of one unit: the sample and four passes, or one pass writing scores.
+__device__ __forceinline__ int chunks_of(const JobDev& J) { return J.mode == 3 ? J.nc : 1 + 4 * J.nc; }
+
 __device__ __forceinline__ void decode(const JobDev& J, int ci, int& pass, int& c)
 {
-    if (ci == 0) {
+    if (J.mode == 3) {
+        pass = kStore;
+        c = ci;
+    } else if (ci == 0) {
         pass = kSamplePass;
         c = 0;
     } else {
@@ -231,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 2) tile_select_kernel(const __grid_c
                 unit_of(P, u, jb, bh, blk);
                 const JobDev& J = P.job[jb];
                 if (J.mode == 0) continue;
-                const int nci = 1 + 4 * J.nc;
+                const int nci = chunks_of(J);
                 for (int ci = 0; ci < nci && ok; ++ci) {
                     int pass, c;
                     decode(J, ci, pass, c);
@@ -266,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 2) tile_select_kernel(const __grid_c
             if (J.mode == 0) continue;
             // the unit's q-hat planes are in TMEM
             if (!(ok = warp_wait(&sm.abort_flag, &sm.a_full, ua & 1, P.status, P.wait_limit))) break;
-            const int nci = 1 + 4 * J.nc;
+            const int nci = chunks_of(J);
             for (int ci = 0; ci < nci && ok; ++ci) {
                 int pass, c;
                 decode(J, ci, pass, c);
@@ -359,7 +365,7 @@ __global__ void __launch_bounds__(kThreads, 2) tile_select_kernel(const __grid_c
                     acc[i] = 0u;
                 }
             };
-            const int nci = 1 + 4 * J.nc;
+            const int nci = chunks_of(J);
             for (int ci = 0; ci < nci; ++ci) {
                 int pass, c;
                 decode(J, ci, pass, c);
@@ -379,7 +385,22 @@ __global__ void __launch_bounds__(kThreads, 2) tile_select_kernel(const __grid_c
                 const bool last = (pass != kSamplePass) && (c == J.nc - 1);
                 bool sort_now = pass == kSamplePass;   // the sample, or the collected band
 
-                if (pass == kCountA || pass == kCountB) {
+                if (pass == kStore) {
+                    // this row's exact scores of the chunk, 16-byte stores (the
+                    // row stride is a multiple of 32 scores)
+                    if (vrow) {
+                        float* dst = J.sc + grow * J.ld + j0;
+                        if (nvalid == kCols) {
+#pragma unroll
+                            for (int e = 0; e < kCols; e += 4)
+                                *reinterpret_cast<uint4*>(dst + e) = make_uint4(sv[e], sv[e + 1], sv[e + 2], sv[e + 3]);
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < kCols; ++e)
+                                if (e < nvalid) dst[e] = __uint_as_float(sv[e]);
+                        }
+                    }
+                } else if (pass == kCountA || pass == kCountB) {
 #pragma unroll
                     for (int e = 0; e < kCols; e += 2) {
                         uint32_t h = g_pair(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1]), scale2, bias2);
@@ -549,7 +570,7 @@ cudaError_t launch_select_tc(const SelectParams& a, cudaStream_t s)
         J.nk = S.nk;
         J.k = S.k;
         J.nc = (S.nk + kCols - 1) / kCols;
-        J.mode = S.k == S.nk ? 0 : 2;
+        J.mode = a.scores_only ? 3 : (S.k == S.nk ? 0 : 2);
         if (J.mode == 2 && !S.k_sample) return cudaErrorInvalidValue;
         J.idx = S.idx;
         J.sc = S.sc;
@@ -558,14 +579,18 @@ cudaError_t launch_select_tc(const SelectParams& a, cudaStream_t s)
         J.first_unit = units;
         units += (int64_t)a.BH * P.n_blk;
         if (!make_plane_map(enc, &P.kmap[jb], S.k_planes, S.nk, 1, S.nk, BH3)) return cudaErrorInvalidValue;
+        if (J.mode == 3 && ((J.ld & 3) != 0 || (reinterpret_cast<uintptr_t>(S.sc) & 15u) != 0))
+            return cudaErrorInvalidValue;
         if (J.mode == 2) {
             // the planes of the 64 sampled key tiles of each head (one box)
             if (!make_plane_map(enc, &P.smap[jb], S.k_sample, kCols, 1, kCols, BH3)) return cudaErrorInvalidValue;
-            cudaError_t e = cudaMemsetAsync(S.fb, 0, sizeof(int32_t), s);
-            if (e != cudaSuccess) return e;
         } else {
             P.smap[jb] = P.kmap[jb];
         }
+        // no row left to the exact top-k yet (the list stays empty unless the
+        // rows are selected on chip)
+        cudaError_t e = cudaMemsetAsync(S.fb, 0, sizeof(int32_t), s);
+        if (e != cudaSuccess) return e;
     }
     P.units = units;
     P.status = a.status;

@@ -92,6 +92,9 @@ struct SelectParams {
     int32_t BH, nq;
     uint32_t* status;
     int32_t short_waits;
+    // 1: only compute the scores (exact, the six plane products) and write
+    // them to each job's `sc`; the caller then runs the top-k kernel
+    int32_t scores_only;
 };
 
 bool select_tc_supported(int r, int n_tiles_max);

@@ -116,7 +116,7 @@ def test_valid_problem_workspace_size(L):
     ({"r": 132}, B.VEDA_ERR_UNSUPPORTED),
     ({"B": 0}, B.VEDA_ERR_INVALID_ARG),
     ({"dtype": 7}, B.VEDA_ERR_INVALID_ARG),
-    ({"flags": 8}, B.VEDA_ERR_INVALID_ARG),
+    ({"flags": 16}, B.VEDA_ERR_INVALID_ARG),
     ({"softmax_scale": -1.0}, B.VEDA_ERR_INVALID_ARG),
     ({"softmax_scale": float("nan")}, B.VEDA_ERR_INVALID_ARG),
     ({"q": 0}, B.VEDA_ERR_INVALID_ARG),
@@ -140,7 +140,8 @@ def test_invalid_arguments_rejected_on_host(L, over, code):
 
 
 def test_test_hook_flags_are_accepted(L):
-    for flags in (B.VEDA_FLAG_SIMT_ATTENTION, B.VEDA_FLAG_TEST_SHORT_WAITS, B.VEDA_FLAG_UNFUSED_SELECTION, 7):
+    for flags in (B.VEDA_FLAG_SIMT_ATTENTION, B.VEDA_FLAG_TEST_SHORT_WAITS, B.VEDA_FLAG_UNFUSED_SELECTION,
+                  B.VEDA_FLAG_ONCHIP_SELECTION, 15):
         st, _ = _ws_size(L, _problem(flags=flags))
         assert st == B.VEDA_OK
 

@@ -1,15 +1,17 @@
-"""The fused tile scoring + top-k (tensor-core scores, on-chip exact
-selection; the default of veda_select_tiles) against the CPU oracle.
+"""Tile selection on the tensor cores against the CPU oracle, in both of its
+forms: tensor-core scores written out and selected by the warp-per-row top-k
+(the default of veda_select_tiles), and the on-chip selection that writes no
+score matrix (VEDA_FLAG_ONCHIP_SELECTION).
 
-  * reduced workloads with more than 128 key tiles (several chunks per row,
-    ragged last chunk and last block of query tiles, a reference segment),
-    budgets 1, ~10 %, n - 1 and n;
+  * reduced workloads with several 64-tile chunks per row (ragged last chunk
+    and last block of query tiles, a reference segment), budgets 1, ~10 %,
+    n - 1 and n;
   * crafted integer scores through the whole pipeline (exact in every
     precision): heavy ties, constant rows, sorted rows, a single winner;
   * rows the on-chip selection cannot finish (all scores equal) go to the
     exact step-3 kernel and still match;
-  * the fused and the three-kernel paths agree outside the tie band, and
-    few rows of a realistic problem need the fallback.
+  * the tensor-core and the fp32 SIMT score paths agree outside the tie band,
+    and few rows of a realistic problem need the on-chip fallback.
 """
 import numpy as np
 import pytest
@@ -53,12 +55,16 @@ def _select(p, g, flags_problem=None):
 MULTI = dict(frames=10, Y=48, X=84, H=4, dense=(("text", 200),))
 
 
+ONCHIP = B.VEDA_FLAG_ONCHIP_SELECTION
+
+
+@pytest.mark.parametrize("flags", [0, ONCHIP], ids=["tensor_scores", "onchip"])
 @pytest.mark.parametrize("budget", [1, 32, 314, 315])
-def test_fused_selection_several_chunks(dev, oracle_mod, budget):
+def test_fused_selection_several_chunks(dev, oracle_mod, budget, flags):
     w = workloads.small("r2va_5.17s", ref_frames=5, budget_video=budget, budget_ref=min(budget, 158), **MULTI)
     inp = workloads.make_inputs(w)
     g = {k: v.to(dev) for k, v in inp.items()}
-    p = _problem(w, g)
+    p = _problem(w, g, flags=flags)
     ws, iv, ir = _select(p, g)
     sel = oracle_mod.select_tiles(inp, w.T, w.budget_video, w.budget_ref)
     rep = compare_selection(oracle_mod, iv.cpu().numpy(), sel["idx_v"], sel["kth_v"], sel["qhat"], sel["khat"])
@@ -66,7 +72,11 @@ def test_fused_selection_several_chunks(dev, oracle_mod, budget):
     rep = compare_selection(oracle_mod, ir.cpu().numpy(), sel["idx_r"], sel["kth_r"], sel["qhat"], sel["khat_r"])
     assert_selection(rep, f"fused k={budget} reference")
     n_rows = w.B * w.H * w.n_q_tiles
-    assert len(veda.fallback_rows(p, ws)) <= max(2, n_rows // 100)
+    fb = len(veda.fallback_rows(p, ws))
+    if flags == 0:
+        assert fb == 0
+    else:   # very small budgets give narrow bands that pass A's approximate scores can miss
+        assert fb <= (n_rows // 6 if budget <= 2 else max(2, n_rows // 50)), fb
 
 
 def _crafted(dev, x, y, a, H=2, T=128):
@@ -91,8 +101,9 @@ def _crafted(dev, x, y, a, H=2, T=128):
     return {"q": q, "k": k, "v": v, "w_q": wmat, "w_k": wmat.clone()}
 
 
+@pytest.mark.parametrize("flags", [0, ONCHIP], ids=["tensor_scores", "onchip"])
 @pytest.mark.parametrize("case", ["ties", "constant", "sorted", "single_winner"])
-def test_fused_selection_crafted_integer_scores(dev, oracle_mod, case):
+def test_fused_selection_crafted_integer_scores(dev, oracle_mod, case, flags):
     rng = np.random.default_rng(3)
     n = 300
     if case == "ties":
@@ -108,7 +119,7 @@ def test_fused_selection_crafted_integer_scores(dev, oracle_mod, case):
     inp = _crafted(dev, x, y, a)
     g = {k_: v_.to(dev) for k_, v_ in inp.items()}
     for k in (1, 7, 30, 150, 299):
-        p = veda.Problem(g["q"], g["k"], g["v"], tile=128, r=64, budget=k)
+        p = veda.Problem(g["q"], g["k"], g["v"], tile=128, r=64, budget=k, flags=flags)
         ws, iv, _ = _select(p, g)
         qhat = oracle_mod.project(oracle_mod.pool(inp["q"], 128), inp["w_q"])
         khat = oracle_mod.project(oracle_mod.pool(inp["k"], 128), inp["w_k"])
@@ -123,22 +134,25 @@ def test_rows_left_to_the_exact_kernel(dev, oracle_mod):
     inp = workloads.make_inputs(w)
     inp["q"] = torch.zeros_like(inp["q"])
     g = {k: v.to(dev) for k, v in inp.items()}
-    p = _problem(w, g)
+    p = _problem(w, g, flags=ONCHIP)
     ws, iv, _ = _select(p, g)
     fb = veda.fallback_rows(p, ws)
     assert len(fb) == w.B * w.H * w.n_q_tiles
     assert (iv.cpu().numpy() == np.arange(20)).all()
 
 
-def test_fused_and_unfused_paths_agree(dev, oracle_mod):
+def test_tensor_simt_and_onchip_paths_agree(dev, oracle_mod):
     w = workloads.small("portrait_10.13s", frames=12, Y=84, X=48, H=4, budget_video=40, dense=())
     inp = workloads.make_inputs(w)
     g = {k: v.to(dev) for k, v in inp.items()}
-    _, iv_f, _ = _select(_problem(w, g), g)
-    _, iv_u, _ = _select(_problem(w, g, flags=B.VEDA_FLAG_UNFUSED_SELECTION), g)
+    _, iv_t, _ = _select(_problem(w, g), g)
+    _, iv_s, _ = _select(_problem(w, g, flags=B.VEDA_FLAG_UNFUSED_SELECTION), g)
+    _, iv_o, _ = _select(_problem(w, g, flags=ONCHIP), g)
     sel = oracle_mod.select_tiles(inp, w.T, w.budget_video)
-    for iv, what in ((iv_f, "fused"), (iv_u, "unfused")):
+    for iv, what in ((iv_t, "tensor scores"), (iv_s, "simt scores"), (iv_o, "on-chip")):
         rep = compare_selection(oracle_mod, iv.cpu().numpy(), sel["idx_v"], sel["kth_v"], sel["qhat"], sel["khat"])
         assert_selection(rep, what)
-    differ = (iv_f != iv_u).any(dim=-1).sum().item()
+    # the same scores, bit for bit: the two tensor-core paths keep the same tiles
+    assert torch.equal(iv_t, iv_o)
+    differ = (iv_t != iv_s).any(dim=-1).sum().item()
     assert differ <= 5, differ
