@@ -90,9 +90,14 @@ struct TcSelParams {
 
 struct __align__(1024) Smem {
     uint8_t kv[kNS][kStageBytes];
-    // band scores, entry e of row t at list[e][t]; entry kCap absorbs the
-    // stores of scores outside the band (branch-free collection)
-    float list[rs::kCap + 1][kRows];
+    union {
+        // band scores, entry e of row t at list[e][t]; entry kCap absorbs the
+        // stores of scores outside the band (branch-free collection)
+        float list[rs::kCap + 1][kRows];
+        // scores-only pass: each warp's 32 rows of a chunk, transposed so the
+        // warp writes whole row segments (rows padded to 68 floats)
+        float stage[4][32][kCols + 4];
+    };
     uint64_t a_full, a_free, kv_full[kNS], kv_empty[kNS], s_full[kNB], s_empty[kNB], drain;
     uint32_t tmem_base;
     volatile int abort_flag;
@@ -386,20 +391,32 @@ __global__ void __launch_bounds__(kThreads, 2) tile_select_kernel(const __grid_c
                 bool sort_now = pass == kSamplePass;   // the sample, or the collected band
 
                 if (pass == kStore) {
-                    // this row's exact scores of the chunk, 16-byte stores (the
-                    // row stride is a multiple of 32 scores)
-                    if (vrow) {
-                        float* dst = J.sc + grow * J.ld + j0;
-                        if (nvalid == kCols) {
+                    // the chunk's exact scores: each thread puts its row in the
+                    // warp's staging area, then the warp writes two rows (256
+                    // contiguous bytes each) per 16-byte store instruction
+                    float(*stg)[kCols + 4] = sm.stage[warp];
 #pragma unroll
-                            for (int e = 0; e < kCols; e += 4)
-                                *reinterpret_cast<uint4*>(dst + e) = make_uint4(sv[e], sv[e + 1], sv[e + 2], sv[e + 3]);
-                        } else {
-#pragma unroll
-                            for (int e = 0; e < kCols; ++e)
-                                if (e < nvalid) dst[e] = __uint_as_float(sv[e]);
+                    for (int e = 0; e < kCols; e += 4)
+                        *reinterpret_cast<uint4*>(&stg[lane][e]) = make_uint4(sv[e], sv[e + 1], sv[e + 2], sv[e + 3]);
+                    __syncwarp();
+                    const int c4 = (lane & 15) * 4;
+#pragma unroll 4
+                    for (int it = 0; it < 16; ++it) {
+                        const int r = 2 * it + (lane >> 4);
+                        const int grow_r = blk * kRows + warp * 32 + r;
+                        if (grow_r < P.nq) {
+                            float* dst = J.sc + ((int64_t)bh * P.nq + grow_r) * J.ld + j0 + c4;
+                            const float4 x = *reinterpret_cast<const float4*>(&stg[r][c4]);
+                            if (c4 + 4 <= nvalid) {
+                                *reinterpret_cast<float4*>(dst) = x;
+                            } else {
+                                if (c4 < nvalid) dst[0] = x.x;
+                                if (c4 + 1 < nvalid) dst[1] = x.y;
+                                if (c4 + 2 < nvalid) dst[2] = x.z;
+                            }
                         }
                     }
+                    __syncwarp();                  // the staging area is reused by the next chunk
                 } else if (pass == kCountA || pass == kCountB) {
 #pragma unroll
                     for (int e = 0; e < kCols; e += 2) {
