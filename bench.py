@@ -62,10 +62,13 @@ def parse():
 
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the
-# attention kernel in its current form, from one ncu capture of 8 of the 32
-# heads of t2v_5.17s (1.6768 GB), scaled by the units processed (x4) to the
-# full launch.  Other workloads have no capture: null.
-ATTN_TRAFFIC = {("t2v_5.17s", 32, 98): 1.6768e9 * 4}
+# attention kernel in its current form (L2 evict-last K/V loads, evict-first
+# Q loads and O stores), from one ncu capture of 8 of the 32 heads of each
+# workload, scaled by the units processed (x4) to the full launch:
+#   t2v_5.17s  1.2719 GB read + 0.2537 GB written = 1.5256 GB (8 heads)
+#   t2v_14.38s 22.7348 GB read + 0.7642 GB written = 23.4990 GB (8 heads)
+# Other workloads have no capture: null.
+ATTN_TRAFFIC = {("t2v_5.17s", 32, 98): 1.5256e9 * 4, ("t2v_14.38s", 32, 138): 23.4990e9 * 4}
 
 
 def peaks():

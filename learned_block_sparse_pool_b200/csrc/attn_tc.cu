@@ -145,9 +145,9 @@ __device__ __forceinline__ bool warp_wait(Smem& sm, uint64_t* b, uint32_t parity
 }
 
 __device__ __forceinline__ void tma_load(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1, int c2,
-                                         int c3)
+                                         int c3, uint64_t policy)
 {
-    tc::tma_load_4d(dst, map, bar, c0, c1, c2, c3);
+    tc::tma_load_4d_hint(dst, map, bar, c0, c1, c2, c3, policy);
 }
 
 #define TMEM_LD32(taddr, r) VEDA_TMEM_LD32(taddr, r)
@@ -243,8 +243,12 @@ __device__ __forceinline__ void load_box_pair(const TcParams& P, int m, uint8_t*
     const int c1 = ph == 1 ? h : (pn == 1 ? tok : b);
     const int c2 = ph == 2 ? h : (pn == 2 ? tok : b);
     const int c3 = ph == 3 ? h : (pn == 3 ? tok : b);
-    tma_load(dst, &P.tm[m], bar, 0, c1, c2, c3);
-    tma_load(dst + kBoxBytes, &P.tm[m], bar, 64, c1, c2, c3);
+    // Q is read by one unit only; a K/V tile is read again by the other query
+    // tiles of its head in flight (head-major unit order), so it stays in L2
+    // ahead of the streaming Q loads and O stores
+    const uint64_t policy = m == 0 ? tc::l2_policy_evict_first() : tc::l2_policy_evict_last();
+    tma_load(dst, &P.tm[m], bar, 0, c1, c2, c3, policy);
+    tma_load(dst + kBoxBytes, &P.tm[m], bar, 64, c1, c2, c3, policy);
 }
 
 // --------------------------------------------------------------- kernel ---
@@ -520,6 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             const int64_t tok = (int64_t)i * TT + row;
             const int64_t prow = kSplit ? (((u % P.n_split) * P.B + b) * (int64_t)P.H + h) * P.n_qtok + tok : 0;
             __nv_bfloat16* dst = P.out + (((int64_t)b * P.n_qtok + tok) * P.H + h) * D + 64 * g;
+            const uint64_t o_policy = tc::l2_policy_evict_first();   // O is written once
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
                 uint32_t o0[32], o1[32];
@@ -558,7 +563,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                         w.y = *reinterpret_cast<uint32_t*>(&v1);
                         w.z = *reinterpret_cast<uint32_t*>(&v2);
                         w.w = *reinterpret_cast<uint32_t*>(&v3);
-                        *reinterpret_cast<uint4*>(dst + 32 * q + c) = w;
+                        tc::st_global_v4_hint(dst + 32 * q + c, w, o_policy);
                     }
                 }
             }
