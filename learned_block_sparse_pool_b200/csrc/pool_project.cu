@@ -60,24 +60,93 @@ __device__ __forceinline__ uint4 load_stream(const void* p)
 }
 
 constexpr int kGroup = 4;   // tiles of one head pooled per round
+constexpr int kWarps = kThreads / 32;
+
+// CTAs per SM the kernel is compiled for: with bf16 rows (8 loads of 16 bytes
+// per thread per tile) it fits 80 registers, so three CTAs per SM keep 1.5x
+// the bytes in flight of two (a 64-register cap for four spills).
+template <typename Tin>
+constexpr int min_blocks() { return sizeof(Tin) == 2 ? 3 : 1; }
+
+// Writes one projected value s = xhat[b, h, tile ti][c] of job J: the fp32
+// output (c < r) and, where the job asks for them, its three bf16 planes
+// (columns r..63 of a plane row are written as zeros) and the sampled tiles'
+// planes.
+__device__ __forceinline__ void store_projection(const PoolParams& P, const PoolJob& J, int bb, int hh, int ti,
+                                                 int c, float s)
+{
+    const int64_t orow = (int64_t)(bb * P.H + hh) * J.n_tiles + ti;
+    if (c < P.r) J.out[orow * P.r + c] = s;
+    if (J.planes) {
+        // three bf16 terms summing to s: each difference is exact in fp32
+        const __nv_bfloat16 p0 = __float2bfloat16_rn(s);
+        const float r1 = s - __bfloat162float(p0);
+        const __nv_bfloat16 p1 = __float2bfloat16_rn(r1);
+        const __nv_bfloat16 p2 = __float2bfloat16_rn(r1 - __bfloat162float(p1));
+        uint16_t* dst = J.planes + orow * kPlaneWidth + c;
+        dst[0] = __bfloat16_as_ushort(p0);
+        dst[J.plane_stride] = __bfloat16_as_ushort(p1);
+        dst[2 * J.plane_stride] = __bfloat16_as_ushort(p2);
+        if (J.sample_planes) {
+            // sample rows m with floor(m n / 64) == this tile: 64 i <= m n < 64 (i + 1)
+            const int64_t n = J.n_tiles;
+            const int64_t m_lo = (64 * (int64_t)ti + n - 1) / n, m_hi = min((int64_t)63, (64 * ((int64_t)ti + 1) + n - 1) / n - 1);
+            for (int64_t m = m_lo; m <= m_hi; ++m) {
+                uint16_t* sd = J.sample_planes + ((int64_t)(bb * P.H + hh) * 64 + m) * kPlaneWidth + c;
+                sd[0] = __bfloat16_as_ushort(p0);
+                sd[J.sample_plane_stride] = __bfloat16_as_ushort(p1);
+                sd[2 * J.sample_plane_stride] = __bfloat16_as_ushort(p2);
+            }
+        }
+    }
+}
+
+// Batch index of a round of ng tiles of job J that ends before item `it`.
+__device__ __forceinline__ int round_batch(const PoolParams& P, const PoolJob& J, int64_t it, int ng)
+{
+    return (int)(((it - ng - J.first_item) / J.n_tiles) / P.H);
+}
+
+// Projection of one round's pooled vectors (ng consecutive tiles i0.. of head
+// hh, the round ending before item `it`): one output (g, c) per thread.
+template <int D>
+__device__ __forceinline__ void project_round(const PoolParams& P, const PoolJob& J, int hh, int64_t it, int ng,
+                                              int i0, const float* w_s, const float* pooled, int tid, int nthreads)
+{
+    const int r = P.r;
+    const int bb = round_batch(P, J, it, ng);
+    const int rc = J.planes ? kPlaneWidth : r;   // columns written per tile
+    for (int x = tid; x < ng * rc; x += nthreads) {
+        const int g = x / rc, c = x % rc;
+        float s = 0.f;
+        if (c < r) {
+            const float* pv = pooled + g * D;
+#pragma unroll 8
+            for (int e = 0; e < D; ++e) s = fmaf(pv[e], w_s[e * r + c], s);
+        }
+        store_projection(P, J, bb, hh, i0 + g, c, s);
+    }
+}
 
 template <typename Tin, int D>
-__global__ void __launch_bounds__(kThreads) pool_project_kernel(const PoolParams P)
+__global__ void __launch_bounds__(kThreads, min_blocks<Tin>()) pool_project_kernel(const PoolParams P)
 {
     constexpr int EPC = 16 / sizeof(Tin);      // elements per 16-byte chunk
-    constexpr int CPR = D / EPC;               // chunks per token row
+    constexpr int CPR = D / EPC;               // chunks per token row (divides 32)
     constexpr int RP = kThreads / CPR;         // token rows loaded in parallel
     constexpr int LOADS = kMaxTile / RP;       // loads per thread per tile (max)
+    static_assert(32 % CPR == 0, "a warp holds whole token rows");
 
     extern __shared__ float smem[];
     const int r = P.r;
     float* w_s = smem;                         // [D][r]
-    float* part = w_s + D * r;                 // [kGroup][RP][D]
-    float* pooled = part + kGroup * RP * D;    // [kGroup][D]
+    float* part = w_s + D * r;                 // [kGroup][kWarps][D]: one partial sum per warp
+    float* pooled = part + kGroup * kWarps * D;   // [kGroup][D]
 
     const int tid = threadIdx.x;
     const int chunk = tid % CPR;
     const int row0 = tid / CPR;
+    const int warp = tid / 32, lane = tid % 32;
 
     const int64_t it0 = (int64_t)blockIdx.x * P.total_items / gridDim.x;
     const int64_t it1 = (int64_t)(blockIdx.x + 1) * P.total_items / gridDim.x;
@@ -147,9 +216,16 @@ __global__ void __launch_bounds__(kThreads) pool_project_kernel(const PoolParams
                 }
             }
             if (it + 1 < it1) issue(P.job[nj], nb, nh, ni);
-            float* dst = part + (g * RP + row0) * D + chunk * EPC;
+            // the lanes of a warp that hold the same column chunk (CPR apart) add up their rows
 #pragma unroll
-            for (int e = 0; e < EPC; ++e) dst[e] = acc[e];
+            for (int off = CPR; off < 32; off <<= 1)
+#pragma unroll
+                for (int e = 0; e < EPC; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
+            if (lane < CPR) {
+                float* dst = part + (g * kWarps + warp) * D + chunk * EPC;
+#pragma unroll
+                for (int e = 0; e < EPC; ++e) dst[e] = acc[e];
+            }
             i = ni; h = nh; b = nb; j = nj;
             ++it;
         }
@@ -160,57 +236,19 @@ __global__ void __launch_bounds__(kThreads) pool_project_kernel(const PoolParams
             const int t0 = (i0 + g) * P.T;
             const int cnt = (int)min((int64_t)P.T, J.n_tokens - (int64_t)t0);
             float s = 0.f;
-#pragma unroll 8
-            for (int q = 0; q < RP; ++q) s += part[(g * RP + q) * D + e];
+#pragma unroll
+            for (int q = 0; q < kWarps; ++q) s += part[(g * kWarps + q) * D + e];
             pooled[g * D + e] = s / (float)cnt;
         }
         __syncthreads();
-        // projection of the round's pooled vectors: one output (g, c) per thread
-        const int hh = cur_h;
-        const int bb = (int)(((it - ng - J.first_item) / J.n_tiles) / P.H);
-        const int rc = J.planes ? kPlaneWidth : r;   // columns written per tile
-        for (int x = tid; x < ng * rc; x += kThreads) {
-            const int g = x / rc, c = x % rc;
-            const int64_t orow = (int64_t)(bb * P.H + hh) * J.n_tiles + i0 + g;
-            float s = 0.f;
-            if (c < r) {
-                const float* pv = pooled + g * D;
-#pragma unroll 8
-                for (int e = 0; e < D; ++e) s = fmaf(pv[e], w_s[e * r + c], s);
-                J.out[orow * r + c] = s;
-            }
-            if (J.planes) {
-                // three bf16 terms summing to s: each difference is exact in fp32
-                const __nv_bfloat16 p0 = __float2bfloat16_rn(s);
-                const float r1 = s - __bfloat162float(p0);
-                const __nv_bfloat16 p1 = __float2bfloat16_rn(r1);
-                const __nv_bfloat16 p2 = __float2bfloat16_rn(r1 - __bfloat162float(p1));
-                uint16_t* dst = J.planes + orow * kPlaneWidth + c;
-                dst[0] = __bfloat16_as_ushort(p0);
-                dst[J.plane_stride] = __bfloat16_as_ushort(p1);
-                dst[2 * J.plane_stride] = __bfloat16_as_ushort(p2);
-                if (J.sample_planes) {
-                    // sample rows m with floor(m n / 64) == this tile: 64 i <= m n < 64 (i + 1)
-                    const int64_t n = J.n_tiles, ti = i0 + g;
-                    const int64_t m_lo = (64 * ti + n - 1) / n, m_hi = min((int64_t)63, (64 * (ti + 1) + n - 1) / n - 1);
-                    for (int64_t m = m_lo; m <= m_hi; ++m) {
-                        uint16_t* sd = J.sample_planes + ((int64_t)(bb * P.H + hh) * 64 + m) * kPlaneWidth + c;
-                        sd[0] = __bfloat16_as_ushort(p0);
-                        sd[J.sample_plane_stride] = __bfloat16_as_ushort(p1);
-                        sd[2 * J.sample_plane_stride] = __bfloat16_as_ushort(p2);
-                    }
-                }
-            }
-        }
+        project_round<D>(P, J, cur_h, it, ng, i0, w_s, pooled, tid, kThreads);
     }
 }
 
 template <typename Tin, int D>
 cudaError_t launch_typed(const PoolParams& p, cudaStream_t s)
 {
-    constexpr int EPC = 16 / sizeof(Tin);
-    constexpr int RP = kThreads / (D / EPC);
-    const size_t smem = sizeof(float) * ((size_t)D * p.r + (size_t)kGroup * RP * D + (size_t)kGroup * D);
+    const size_t smem = sizeof(float) * ((size_t)D * p.r + (size_t)kGroup * kWarps * D + (size_t)kGroup * D);
     auto kern = pool_project_kernel<Tin, D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
