@@ -4,8 +4,14 @@
 // the top `budget` (tao.media, "Affine launches MiniMax-H3 video studio...",
 // sections "Training the Selector, Not the Generator" and "How the SN120
 // Competition Works"; reference and video tiles are selected independently:
-// veyrul.com, "Veda R2VA for MiniMax-H3", second paragraph).  This kernel does
-// both steps without ever writing the score matrix to memory:
+// veyrul.com, "Veda R2VA for MiniMax-H3", second paragraph).  It runs in one
+// of two modes:
+//   scores only (the default selection path): the tensor-core scores of each
+//     chunk are staged through shared memory (a per-warp transpose) and
+//     written to the workspace's score matrix in coalesced rows; the
+//     warp-per-row top-k then selects from them;
+//   on chip: both steps without ever writing the score matrix to memory, as
+//     follows.
 //
 //   scores  s[i][j] = qhat_i . khat_j on the tensor cores.  The pool +
 //           project kernel writes each projection as three bf16 planes
