@@ -2,9 +2,9 @@
 """Benchmark of the Veda-style block-sparse attention hot path on B200.
 
 One step = one full pass of the path over one synthetic layer call:
-tile pool + selector projection -> tile scores + fixed-budget top-k (fused on
-the tensor cores) -> block-sparse attention (the stages veda_attn runs),
-inputs resident in HBM.  Default workload: the 1344x768, 24 fps, 5.17 s landscape clip
+tile pool + selector projection -> tile scores (tensor cores) + fixed-budget
+top-k -> block-sparse attention (the stages veda_attn runs), inputs resident
+in HBM.  Default workload: the 1344x768, 24 fps, 5.17 s landscape clip
 (31 x 48 x 84 = 124,992 video tokens, 32 heads, head dim 128, tile 128,
 90% sparsity = 98 kept tiles, 512 text + 256 audio dense keys), bf16.
 
