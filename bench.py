@@ -11,14 +11,17 @@ in HBM.  Default workload: the 1344x768, 24 fps, 5.17 s landscape clip
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...   (times the CPU oracle instead)
 
-Prints one JSON line on rank 0.  Multi-GPU (torchrun): every rank runs its
-own independent layer call (weak scaling, no data-path collective); the
-timed region is bracketed by barriers and the max over ranks is reported.
+Prints one JSON line on rank 0.  Multi-GPU (torchrun): by default every rank
+runs its own independent layer call (weak scaling); with --split heads the
+heads of one call are split into contiguous ranges, one per rank (strong
+scaling).  Neither has a data-path collective; the timed region is bracketed
+by barriers and the max over ranks is reported.
 """
 from __future__ import annotations
 
 import argparse
 import atexit
+import dataclasses
 import datetime
 import json
 import os
@@ -53,6 +56,9 @@ def parse():
                     help="time the three-kernel selection (fp32 SIMT scores, then the warp-per-row top-k)")
     ap.add_argument("--onchip-selection", action="store_true",
                     help="time the on-chip selection (tensor-core scores recomputed per pass, no score matrix)")
+    ap.add_argument("--split", choices=["calls", "heads"], default="calls",
+                    help="N GPUs: one independent layer call per GPU (weak scaling), or the heads of one "
+                         "call split into N contiguous ranges, no collective (strong scaling)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ncu", action="store_true", help="short run for profiler captures (no extras)")
@@ -208,11 +214,26 @@ def max_over_ranks(dist, values, device):
     return t.tolist()
 
 
-def bench_config(w, n, simt=False):
+def head_range(H, n, rank):
+    """Heads [h0, h1) of `rank` when the H heads of one call are split into n
+    contiguous, near-equal ranges (every head is an independent problem)."""
+    return rank * H // n, (rank + 1) * H // n
+
+
+def head_slice(g, h0, h1):
+    """The inputs of heads [h0, h1): strided views of the [B, N, H, d]
+    tensors (the library takes any 16-byte strides) and of the [H, d, r]
+    selector weights."""
+    return {k: (v[h0:h1] if k in ("w_q", "w_k") else v[:, :, h0:h1]) for k, v in g.items()}
+
+
+def bench_config(w, n, simt=False, split="calls"):
     """The `config` object of the JSON line (identical in both arms)."""
+    par = (f"{n} independent layer calls (one per GPU)" if split == "calls" or n == 1 else
+           f"the {w.H} heads of one call split over {n} GPUs (contiguous ranges, no collective)")
     return dict(w.describe(), **{
         "kept_tflop_per_call": round(w.kept_flops() / 1e12, 3),
-        "parallelism": f"{n} independent layer calls (one per GPU)",
+        "parallelism": par,
         "l2": "inputs larger than L2 (Q, K, V of one call exceed 126 MB each)",
         "attention_kernel": "simt" if (simt or w.dtype != "bf16") else "tcgen05",
     })
@@ -262,9 +283,20 @@ def main():
     g = workloads.make_inputs(w, device=dev)
     sel_flags = (veda.binding.VEDA_FLAG_UNFUSED_SELECTION if args.unfused_selection else 0) | \
         (veda.binding.VEDA_FLAG_ONCHIP_SELECTION if args.onchip_selection else 0)
-    p = make_problem(veda, w, g, args.simt, sel_flags)
+    # calls: every rank runs the whole call (n calls per step); heads: every
+    # rank runs its head range of the same call (one call per step)
+    split = args.split == "heads" and n > 1
+    calls_per_step = 1 if split else n
+    w_run = w
+    if split:
+        h0, h1 = head_range(w.H, n, rank)
+        g = head_slice(g, h0, h1)
+        w_run = dataclasses.replace(w, H=h1 - h0)
+    p = make_problem(veda, w_run, g, args.simt, sel_flags)
     ws = veda.workspace(p)
     if args.dense_queries:
+        if split:
+            raise SystemExit("--dense-queries runs whole calls (--split calls)")
         dense_query_run(args, veda, w, g, p, ws, dev, local, rank, n, dist)
         return
     iv, ir = veda.alloc_indices(p)
@@ -327,8 +359,10 @@ def main():
     st_ms = {name: stage_avg[i] for i, (name, _) in enumerate(stages)}
 
     pk, pk_src = peaks()
+    # per-GPU work: the whole call, or (heads split) the largest rank's share
+    wm = dataclasses.replace(w, H=-(-w.H // n)) if split else w
     attn_s = st_ms["attention"] / 1e3
-    flops = w.kept_flops()
+    flops = wm.kept_flops()
     achieved_tf = flops / attn_s / 1e12
     sustained_tf = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     burst_tf = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
@@ -337,16 +371,16 @@ def main():
     long_region = total_ms > 5000.0
     peak_tf = sustained_tf if long_region else burst_tf
     hbm = pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-    esz = 2 if w.dtype == "bf16" else 4
-    pool_bytes = (2 * w.n_video + w.n_ref) * w.B * w.H * w.d * esz
-    rows = w.B * w.H * w.n_q_tiles
+    esz = 2 if wm.dtype == "bf16" else 4
+    pool_bytes = (2 * wm.n_video + wm.n_ref) * wm.B * wm.H * wm.d * esz
+    rows = wm.B * wm.H * wm.n_q_tiles
     selector = {
         "pool_project_gbs": round(pool_bytes / (st_ms["pool_project"] / 1e3) / 1e9, 1),
         "pool_project_frac": round(pool_bytes / (st_ms["pool_project"] / 1e3) / 1e9 / hbm, 4),
         "peak_gbs": hbm, "peak_kind": f"HBM copy ({pk_src})",
     }
-    segs = [(w.n_q_tiles, w.budget_video)] + ([(w.n_ref_tiles, w.budget_ref)] if w.ref_frames else [])
-    score_flop = sum(2.0 * w.r * rows * nk for nk, _ in segs)
+    segs = [(wm.n_q_tiles, wm.budget_video)] + ([(wm.n_ref_tiles, wm.budget_ref)] if wm.ref_frames else [])
+    score_flop = sum(2.0 * wm.r * rows * nk for nk, _ in segs)
     if args.unfused_selection:
         # a row's scores are read unless every tile is kept; the kept indices are written
         topk_bytes = sum(rows * ((nk * 4 if k < nk else 0) + k * 4) for nk, k in segs)
@@ -384,24 +418,25 @@ def main():
 
     res = {
         "metric": METRIC,
-        "value": round(total_ms / args.steps / n, 4),
+        "value": round(total_ms / args.steps / calls_per_step, 4),
         "unit": "ms",
         "n_gpus": n,
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": round(total_ms / args.steps, 4),
         "higher_is_better": False,
-        "scaling": "weak",
+        "scaling": "strong" if split else "weak",
         "vs_baseline": None,
         "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic (seeded; N(0,1) + smooth sinusoid component, shapes of the 1344x768 24 fps clips)",
-        "config": bench_config(w, n, args.simt),
+        "config": bench_config(w, n, args.simt, args.split),
         "kernels_ms": {name: round(v, 4) for name, v in st_ms.items()},
         "roofline": {
             "kernel": "block-sparse attention",
             "bound": "tensor", "achieved": round(achieved_tf, 2), "peak": peak_tf, "unit": "TFLOP/s",
             "frac": round(achieved_tf / peak_tf, 4),
-            "traffic": ATTN_TRAFFIC.get((w.name, w.H, w.budget_video)),
+            "traffic": (None if (w.name, w.H, w.budget_video) not in ATTN_TRAFFIC else
+                        ATTN_TRAFFIC[(w.name, w.H, w.budget_video)] * wm.H / w.H),
             "peak_kind": (f"bf16 dense, {'sustained' if long_region else 'burst'} ({pk_src}; timed region "
                           f"{total_ms / 1e3:.2f} s)"),
             "frac_of_burst_peak": round(achieved_tf / burst_tf, 4),
@@ -414,7 +449,7 @@ def main():
     }
 
     if not args.ncu and not args.no_e2e:
-        res["e2e"] = e2e_run(veda, w, g, p, dev, stream, args.steps, n, dist, args.simt)
+        res["e2e"] = e2e_run(veda, w_run, g, p, dev, stream, args.steps, calls_per_step, dist, args.simt)
     if not args.ncu and not args.no_cpu_baseline and n == 1 and rank == 0:
         ms, cores, sample = oracle_sample(w, host_copy(g), oracle_units(w))
         res["cpu_baseline"] = {"value": round(ms, 1), "unit": "ms", "cores": cores, "kind": "oracle",
@@ -488,7 +523,7 @@ def dense_query_run(args, veda, w, g, p, ws, dev, local, rank, n, dist):
         dist.destroy_process_group()
 
 
-def e2e_run(veda, w, g, p, dev, stream, steps, n, dist, simt, heads_per_group=2):
+def e2e_run(veda, w, g, p, dev, stream, steps, calls_per_step, dist, simt, heads_per_group=2):
     """Same metric through the public host-buffer call (veda_attn_host): every
     step takes Q, K, V, the dense and reference keys and the selector weights
     from pinned host memory and returns the attention output to pinned host
@@ -520,7 +555,8 @@ def e2e_run(veda, w, g, p, dev, stream, steps, n, dist, simt, heads_per_group=2)
     st = veda.check_status(buf, stream)
     if st != 0:
         raise RuntimeError(f"device status after e2e: {veda.status_string(st)}")
-    return {"value": round(ms / k2 / n, 4), "unit": "ms", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+    return {"value": round(ms / k2 / calls_per_step, 4), "unit": "ms", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h,
             "steps": k2, "call": f"veda_attn_host (pinned host buffers, {heads_per_group} heads per group)"}
 
 
@@ -546,7 +582,7 @@ def run_reference(args, w, dev, n):
         "metric": METRIC, "value": round(v, 1), "unit": "ms", "n_gpus": n, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(wall / args.steps * 1e3, 1), "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": bench_config(w, n, args.simt),
+        "config": bench_config(w, n, args.simt, args.split),
         "cpu_baseline": {"value": round(v, 1), "unit": "ms", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": round(v, 1), "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
