@@ -31,3 +31,23 @@ def oracle_mod():
         assert oracle.__file__.startswith(_ALT_ORACLE), oracle.__file__
     oracle.build()
     return oracle
+
+
+# Parity reports (selection rows that differ from the oracle only inside the
+# tie band; rows the on-chip selection left to the exact kernel) are emitted
+# as TieBandReport warnings by tests/parity.py and the GPU parity tests; they
+# are gathered here and repeated as one section at the end of the run, just
+# above the final counts, so that a short tail of the log shows them.
+_PARITY_REPORTS = []
+
+
+def pytest_warning_recorded(warning_message, when, nodeid, location):
+    if warning_message.category.__name__ == "TieBandReport":
+        _PARITY_REPORTS.append(str(warning_message.message))
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    if _PARITY_REPORTS:
+        terminalreporter.section("parity reports (tie band; rows finished by the exact kernel)")
+        for line in _PARITY_REPORTS:
+            terminalreporter.write_line(line)
