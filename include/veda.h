@@ -84,12 +84,15 @@ typedef enum { VEDA_F32 = 0, VEDA_BF16 = 1 } veda_dtype;
                                        where the tensor-core kernel applies (bf16,
                                        d = 128, tile = 128): a cross-check path  */
 #define VEDA_FLAG_TEST_SHORT_WAITS 2u /* test hook for the failure path: the
-                                       tensor-core attention kernel's pipeline
-                                       waits give up after ~64 clocks, so the
-                                       call stops early, frees its resources and
-                                       reports VEDA_ERR_TIMEOUT through
+                                       pipeline waits of the tensor-core kernels
+                                       (attention, tile selection) give up after
+                                       ~64 clocks, so the call stops early,
+                                       frees its resources and reports
+                                       VEDA_ERR_TIMEOUT through
                                        veda_check_status(); its output is then
-                                       undefined.  No effect on other kernels. */
+                                       undefined.  No effect on the kernels
+                                       without waits (pool + project, SIMT
+                                       score, top-k, SIMT attention). */
 #define VEDA_FLAG_UNFUSED_SELECTION 4u /* compute the tile scores with the fp32
                                        SIMT kernel instead of the tensor cores
                                        (a cross-check path; also used when
