@@ -356,6 +356,32 @@ def test_full_size_workload(dev, oracle_mod, name):
     print(f"{name}: attention on {len(units)} units: max-abs {err[0]:.3g} rel-L2 {err[1]:.3g}")
 
 
+# The fused on-chip selection (score + top-k in one kernel, no score matrix
+# in HBM) at full size: every row against the oracle, and the rows it hands to
+# the exact kernel bounded: at most 1%, except on the portrait clip, whose
+# +3-boosted key tiles (most likely) stretch the sampled score range and so coarsen the
+# fp16 map that places each row's band (measured: 9,325 of 76,880 rows, 12%).
+ONCHIP_FALLBACK_MAX = {"portrait_10.13s": 0.15}
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_onchip_selection(dev, oracle_mod, name):
+    w = workloads.get(name)
+    g = workloads.make_inputs(w, device=dev)
+    p = make_problem(w, g, flags=veda.binding.VEDA_FLAG_ONCHIP_SELECTION)
+    ws = veda.workspace(p)
+    iv, ir = gpu_select(p, g, ws)
+    torch.cuda.synchronize()
+    assert veda.check_status(ws) == 0
+    host = {k: v.cpu() for k, v in g.items()}
+    sel = oracle_mod.select_tiles(host, w.T, w.budget_video, w.budget_ref if w.ref_frames else 0)
+    rep = check_selection(oracle_mod, p, ws, iv, ir, sel, name + " on chip", host)
+    _report(name + " on chip", rep)
+    fb = len(veda.fallback_rows(p, ws))
+    warnings.warn(f"{name} on chip: {fb} of {rep.rows} rows finished by the exact step-3 kernel", TieBandReport)
+    assert fb <= rep.rows * ONCHIP_FALLBACK_MAX.get(name, 0.01)
+
+
 # The 14.38 s clip's budget sweep (80 / 90 / 98 % sparsity; 95 % is the
 # workload's own budget above) and the portrait clip's dense denominator
 # (budget = every tile): selection on every row, attention on sampled units
