@@ -22,6 +22,16 @@ MUTANTS = {
     "project_transposed_weight": ("(h * d + e) * r + c)", "(h * r + c) * d + e)"),
     "project_ignores_head": ("(h * d + e) * r + c)", "(e) * r + c)"),
     "score_uses_query_twice": ("acc += q[c] * k[c];", "acc += q[c] * q[c];"),
+    "score_keys_of_head_zero": ("const double* k = khat + ((b * H + h) * nk + j) * r;",
+                                "const double* k = khat + ((b * H + 0) * nk + j) * r;"),
+    "select_kth_score_one_rank_early": ("if (kth) kth[rid] = row[k - 1].s;",
+                                        "if (kth) kth[rid] = row[k > 1 ? k - 2 : 0].s;"),
+    "score_keys_of_batch_zero": ("const double* k = khat + ((b * H + h) * nk + j) * r;",
+                                 "const double* k = khat + ((0 * H + h) * nk + j) * r;"),
+    "pool_reads_head_zero": ("o[e] += elem(x, dtype, b * sb + t * st + h * sh + e);",
+                             "o[e] += elem(x, dtype, b * sb + t * st + e);"),
+    "attend_values_of_head_zero": ("o[e] += w * elem(s->v, p->dtype, base + e);",
+                                   "o[e] += w * elem(s->v, p->dtype, base - h * s->sh + e);"),
     "select_keeps_lowest_scores": ("if (a->s > b->s) return -1;\n    if (a->s < b->s) return 1;",
                                    "if (a->s < b->s) return -1;\n    if (a->s > b->s) return 1;"),
     "select_ties_to_highest_index": ("return (a->j > b->j) - (a->j < b->j);",

@@ -199,6 +199,28 @@ def test_select_bruteforce_subsets(oracle_mod):
         assert idx.reshape(-1).tolist() == list(best), (s, k)
 
 
+def test_select_planted_per_head(oracle_mod):
+    """Several heads with their own planted integer scores (q-hat = e_0 in
+    every head, k-hat_j = s_hj e_0): each head's kept set is its own
+    brute-force best k-subset, so a score or selection that mixes heads
+    (or batch entries) fails."""
+    rng = np.random.default_rng(23)
+    B, H, n = 2, 3, 7
+    s = rng.integers(-4, 5, size=(B, H, n)).astype(float)
+    s[0, 1] = s[0, 0][::-1]                 # heads with permuted scores: a head mix-up changes the set
+    qhat = np.zeros((B, H, 1, 2))
+    qhat[..., 0] = 1.0
+    khat = np.zeros((B, H, n, 2))
+    khat[..., 0] = s
+    for k in (1, 3, 6):
+        idx, kth, _ = oracle_mod.select(qhat, khat, k)
+        for b, h in itertools.product(range(B), range(H)):
+            best = max(itertools.combinations(range(n), k),
+                       key=lambda c: (sum(s[b, h, j] for j in c), -sum(c)))
+            assert idx[b, h, 0].tolist() == list(best), (b, h, k)
+            assert kth[b, h, 0] == sorted(s[b, h])[::-1][k - 1]
+
+
 def test_select_properties_random(oracle_mod):
     rng = np.random.default_rng(5)
     B, H, nq, nk, r = 2, 3, 9, 23, 4
