@@ -32,6 +32,12 @@ MUTANTS = {
                              "o[e] += elem(x, dtype, b * sb + t * st + e);"),
     "attend_values_of_head_zero": ("o[e] += w * elem(s->v, p->dtype, base + e);",
                                    "o[e] += w * elem(s->v, p->dtype, base - h * s->sh + e);"),
+    "select_next_equals_kth": ("if (next) next[rid] = (k < nk) ? row[k].s : NAN;",
+                               "if (next) next[rid] = (k < nk) ? row[k - 1].s : NAN;"),
+    "attend_lse_base_two": ("if (lse) lse[u * T + tt] = mx + log(z);",
+                            "if (lse) lse[u * T + tt] = mx + log2(z);"),
+    "pool_token_and_head_strides_swapped": ("o[e] += elem(x, dtype, b * sb + t * st + h * sh + e);",
+                                            "o[e] += elem(x, dtype, b * sb + t * sh + h * st + e);"),
     "select_keeps_lowest_scores": ("if (a->s > b->s) return -1;\n    if (a->s < b->s) return 1;",
                                    "if (a->s < b->s) return -1;\n    if (a->s > b->s) return 1;"),
     "select_ties_to_highest_index": ("return (a->j > b->j) - (a->j < b->j);",
@@ -77,6 +83,10 @@ PY_MUTANTS = {
         'select(qhat, khat_r, budget_ref)', 'select(qhat, khat, budget_ref)'),
     "select_tiles_reference_with_video_budget": (
         'select(qhat, khat_r, budget_ref)', 'select(qhat, khat_r, budget_video)'),
+    "select_tiles_video_keys_projected_with_wq": (
+        'khat = project(pool(inp["k"], T), inp["w_k"])', 'khat = project(pool(inp["k"], T), inp["w_q"])'),
+    "select_tiles_queries_projected_with_wk": (
+        'qhat = project(pool(inp["q"], T), inp["w_q"])', 'qhat = project(pool(inp["q"], T), inp["w_k"])'),
 }
 
 
