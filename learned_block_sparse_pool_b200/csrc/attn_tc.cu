@@ -15,7 +15,10 @@
 //   warp 8      TMA producer: the Q tile and a 5-stage ring of 32 KB K/V
 //               tiles, loaded in exactly the order the MMA warp consumes
 //               them: K0, K1, V0, K2, V1, ..., V(n-1).  Each tile is two
-//               128-row x 128-byte boxes with the 128-byte swizzle.
+//               128-row x 128-byte boxes with the 128-byte swizzle.  K/V
+//               loads carry an L2 evict-last policy (the other query tiles
+//               of the head read them again), Q loads and the O stores an
+//               evict-first one.
 //   warp 9      allocates TMEM and issues the MMAs (the warp runs the loop,
 //               one elected lane issues).  Kept tile j goes to softmax group
 //               g = j & 1: S(j) = Q K(j)^T into S buffer g, then
