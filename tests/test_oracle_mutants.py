@@ -87,6 +87,12 @@ PY_MUTANTS = {
         'khat = project(pool(inp["k"], T), inp["w_k"])', 'khat = project(pool(inp["k"], T), inp["w_q"])'),
     "select_tiles_queries_projected_with_wk": (
         'qhat = project(pool(inp["q"], T), inp["w_q"])', 'qhat = project(pool(inp["q"], T), inp["w_k"])'),
+    "attend_units_reference_keys_and_values_swapped": (
+        'ref = (inp["k_ref"], inp["v_ref"]) if ("k_ref" in inp and idx_r is not None) else None',
+        'ref = (inp["v_ref"], inp["k_ref"]) if ("k_ref" in inp and idx_r is not None) else None'),
+    "attend_units_dense_keys_and_values_swapped": (
+        'dense = (inp["k_dense"], inp["v_dense"]) if "k_dense" in inp else None\n    return attend(inp["q"]',
+        'dense = (inp["v_dense"], inp["k_dense"]) if "k_dense" in inp else None\n    return attend(inp["q"]'),
 }
 
 

@@ -332,7 +332,10 @@ def test_attend_full_budget_is_dense_attention(oracle_mod, dtype):
         np.testing.assert_allclose(lse[u, :c], want_lse, rtol=1e-12, atol=1e-12)
 
 
-def test_attend_masked_dense_equivalence_with_reference_segment(oracle_mod):
+@pytest.mark.parametrize("via", ["attend", "attend_units"])
+def test_attend_masked_dense_equivalence_with_reference_segment(oracle_mod, via):
+    """Through attend() and through attend_units(), the composition the GPU
+    parity tests call with a problem's tensors."""
     B, H, d, T = 1, 2, 8, 4
     N, Nr, Nd = 30, 13, 6
     p = _problem(2, B, H, d, T, N, n_ref=Nr, n_dense=Nd)
@@ -347,9 +350,12 @@ def test_attend_masked_dense_equivalence_with_reference_segment(oracle_mod):
     idx_v[0, 0, 0] = [0, 5, 7]
     idx_r[0, 0, 0] = [1, 3]
     units = [(0, h, i) for h in range(H) for i in range(nq)]
-    out, lse = oracle_mod.attend(p["q"], (p["k"], p["v"]), T, idx_v, units,
-                                 ref=(p["k_ref"], p["v_ref"]), idx_r=idx_r,
-                                 dense=(p["k_dense"], p["v_dense"]), scale=0.3)
+    if via == "attend":
+        out, lse = oracle_mod.attend(p["q"], (p["k"], p["v"]), T, idx_v, units,
+                                     ref=(p["k_ref"], p["v_ref"]), idx_r=idx_r,
+                                     dense=(p["k_dense"], p["v_dense"]), scale=0.3)
+    else:
+        out, lse = oracle_mod.attend_units(p, T, idx_v, idx_r, units, scale=0.3)
     for u, (b, h, i) in enumerate(units):
         qs = p["q"][b, i * T:min(N, (i + 1) * T), h].double()
         keys = torch.cat([p["k"][b, :, h], p["k_ref"][b, :, h], p["k_dense"][b, :, h]]).double()
