@@ -90,6 +90,8 @@ PY_MUTANTS = {
     "attend_units_reference_keys_and_values_swapped": (
         'ref = (inp["k_ref"], inp["v_ref"]) if ("k_ref" in inp and idx_r is not None) else None',
         'ref = (inp["v_ref"], inp["k_ref"]) if ("k_ref" in inp and idx_r is not None) else None'),
+    "attend_dense_queries_skip_reference": (
+        '    ref, idx_r = None, None\n    if "k_ref" in inp:', '    ref, idx_r = None, None\n    if False:'),
     "attend_units_dense_keys_and_values_swapped": (
         'dense = (inp["k_dense"], inp["v_dense"]) if "k_dense" in inp else None\n    return attend(inp["q"]',
         'dense = (inp["v_dense"], inp["k_dense"]) if "k_dense" in inp else None\n    return attend(inp["q"]'),
