@@ -4,11 +4,13 @@ Each case copies the oracle (oracle/veda_oracle.c, or the Python package that
 composes its steps, oracle/__init__.py), plants one mistake (a dropped term, a
 wrong index, a reversed comparison, a swapped operand, ...), builds the copy on
 the CPU and runs the pin suite against it: the suite has to fail.  The
-committed oracle is never modified.
+committed oracle is never modified.  The selected cases run concurrently
+(each is its own build and pytest process); each test reports its own case.
 """
 import os
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 import pytest
 
@@ -57,8 +59,14 @@ MUTANTS = {
 }
 
 
-@pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_pins_catch_planted_mistake(name, tmp_path):
+def _run_pins(env):
+    return subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                           os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                          cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
+
+
+def _c_mutant(name, tmp_path):
+    """Build the C oracle with mistake `name` and run the pins against it."""
     old, new = MUTANTS[name]
     src = open(SRC).read()
     assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
@@ -67,11 +75,8 @@ def test_pins_catch_planted_mistake(name, tmp_path):
     so = tmp_path / "libmutant.so"
     subprocess.run(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-ffp-contract=off",
                     "-o", str(so), str(mutant), "-lm"], check=True)
-    env = dict(os.environ, VEDA_ORACLE_LIB=str(so), OMP_NUM_THREADS="2")
-    res = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                          os.path.join(ROOT, "tests", "test_oracle_pins.py")],
-                         cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
-    assert res.returncode != 0, f"pins did not catch mutant {name}:\n{res.stdout[-2000:]}"
+    env = dict(os.environ, VEDA_ORACLE_LIB=str(so), OMP_NUM_THREADS="1")
+    return _run_pins(env)
 
 
 # Mistakes in the Python composition of the steps (oracle/__init__.py).
@@ -98,8 +103,9 @@ PY_MUTANTS = {
 }
 
 
-@pytest.mark.parametrize("name", sorted(PY_MUTANTS))
-def test_pins_catch_planted_mistake_in_composition(name, tmp_path):
+def _py_mutant(name, tmp_path):
+    """A copy of the oracle package with mistake `name` in its Python
+    composition, ahead of the repository's on sys.path; the pins run on it."""
     old, new = PY_MUTANTS[name]
     src = open(PY).read()
     assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
@@ -108,13 +114,51 @@ def test_pins_catch_planted_mistake_in_composition(name, tmp_path):
     (pkg / "__init__.py").write_text(src.replace(old, new))
     (pkg / "veda_oracle.c").write_text(open(SRC).read())
     # tests/conftest.py puts VEDA_ORACLE_DIR ahead of the repository on sys.path
-    env = dict(os.environ, VEDA_ORACLE_DIR=str(tmp_path), OMP_NUM_THREADS="2")
+    env = dict(os.environ, VEDA_ORACLE_DIR=str(tmp_path), OMP_NUM_THREADS="1")
     env.pop("VEDA_ORACLE_LIB", None)
     probe = subprocess.run([sys.executable, "-c", "import sys; sys.path.insert(0, %r); "
                             "sys.path.insert(0, %r); import oracle; print(oracle.__file__)" % (ROOT, str(tmp_path))],
                            cwd=ROOT, env=env, capture_output=True, text=True, check=True)
     assert probe.stdout.strip().startswith(str(tmp_path)), probe.stdout
-    res = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                          os.path.join(ROOT, "tests", "test_oracle_pins.py")],
-                         cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    return _run_pins(env)
+
+
+C_TEST = "test_pins_catch_planted_mistake"
+PY_TEST = "test_pins_catch_planted_mistake_in_composition"
+
+
+@pytest.fixture(scope="module")
+def mutant_runs(request, tmp_path_factory):
+    """Every selected mutant of this module, run concurrently (each is an
+    independent build and pytest process); results keyed by (test, name)."""
+    jobs = [(item.originalname, item.callspec.params["name"]) for item in request.session.items
+            if item.module is request.module and hasattr(item, "callspec")]
+    run = {C_TEST: _c_mutant, PY_TEST: _py_mutant}
+    # folders made here, one after another (mktemp is not safe across threads)
+    dirs = [tmp_path_factory.mktemp(name) for _, name in jobs]
+
+    def one(job_dir):
+        (test, name), d = job_dir
+        try:
+            return run[test](name, d)
+        except Exception as e:          # reported by the test that owns the job
+            return e
+
+    with ThreadPoolExecutor(max_workers=max(1, min(8, os.cpu_count() or 1))) as ex:
+        return dict(zip(jobs, ex.map(one, zip(jobs, dirs))))
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(name, mutant_runs):
+    res = mutant_runs[(C_TEST, name)]
+    if isinstance(res, Exception):
+        raise res
+    assert res.returncode != 0, f"pins did not catch mutant {name}:\n{res.stdout[-2000:]}"
+
+
+@pytest.mark.parametrize("name", sorted(PY_MUTANTS))
+def test_pins_catch_planted_mistake_in_composition(name, mutant_runs):
+    res = mutant_runs[(PY_TEST, name)]
+    if isinstance(res, Exception):
+        raise res
     assert res.returncode != 0, f"pins did not catch mutant {name}:\n{res.stdout[-2000:]}"
