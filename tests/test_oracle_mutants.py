@@ -19,6 +19,11 @@ SRC = os.path.join(ROOT, "oracle", "veda_oracle.c")
 PY = os.path.join(ROOT, "oracle", "__init__.py")
 
 MUTANTS = {
+    "score_drops_last_component": ("for (int64_t c = 0; c < r; ++c) acc += q[c] * k[c];",
+                                   "for (int64_t c = 0; c < r - 1; ++c) acc += q[c] * k[c];"),
+    "score_components_misaligned": ("for (int64_t c = 0; c < r; ++c) acc += q[c] * k[c];",
+                                    "for (int64_t c = 0; c < r; ++c) acc += q[c] * k[(c + 1) % r];"),
+    "attend_lse_without_max": ("if (lse) lse[u * T + tt] = mx + log(z);", "if (lse) lse[u * T + tt] = log(z);"),
     "pool_divides_by_T": ("o[e] = o[e] / (double)c;", "o[e] = o[e] / (double)T;"),
     "pool_tile_end_off_by_one": ("int64_t t1 = min64(N, t0 + T);", "int64_t t1 = min64(N, t0 + T - 1);"),
     "project_transposed_weight": ("(h * d + e) * r + c)", "(h * r + c) * d + e)"),
