@@ -100,6 +100,14 @@ PY_MUTANTS = {
     "attend_units_reference_keys_and_values_swapped": (
         'ref = (inp["k_ref"], inp["v_ref"]) if ("k_ref" in inp and idx_r is not None) else None',
         'ref = (inp["v_ref"], inp["k_ref"]) if ("k_ref" in inp and idx_r is not None) else None'),
+    "pool_wrapper_token_and_head_strides_swapped": (
+        "lib().oracle_pool(x.data_ptr(), _code(x), B, N, H, d, sb, st, sh, T, _ptr(out))",
+        "lib().oracle_pool(x.data_ptr(), _code(x), B, N, H, d, sb, sh, st, T, _ptr(out))"),
+    "attend_default_scale_one_over_d": (
+        "p.scale = (1.0 / math.sqrt(d)) if scale is None else float(scale)",
+        "p.scale = (1.0 / d) if scale is None else float(scale)"),
+    "attend_query_strides_from_video_keys": (
+        "p.qsb, p.qst, p.qsh, _ = q.stride()", "p.qsb, p.qst, p.qsh, _ = _cpu(video[0]).stride()"),
     "attend_dense_queries_skip_reference": (
         '    ref, idx_r = None, None\n    if "k_ref" in inp:', '    ref, idx_r = None, None\n    if False:'),
     "attend_units_dense_keys_and_values_swapped": (
